@@ -1,0 +1,43 @@
+"""Seeded generators: deterministic, right shapes, planted structure present."""
+import math
+
+import torch
+
+import workloads
+
+
+def test_deterministic_and_shapes():
+    for idx in range(5):
+        w = workloads.get(idx)
+        small = w.with_(L=max(w.B * 4, w.frame_len * 2 if w.recipe == "video" else 0))
+        a, b = workloads.generate(small, seed=0), workloads.generate(small, seed=0)
+        for k in "QKV":
+            assert torch.equal(a[k].view(torch.int16), b[k].view(torch.int16))
+            assert a[k].dtype == torch.bfloat16 and a[k].is_contiguous()
+        assert a["Q"].shape == (w.H, small.L, w.d)
+        assert a["K"].shape == (w.Hkv, small.L, w.d) == a["V"].shape
+        c = workloads.generate(small, seed=1)
+        assert not torch.equal(a["Q"].view(torch.int16), c["Q"].view(torch.int16))
+
+
+def test_sinks_and_ar_correlation():
+    w = workloads.get(0)
+    t = workloads.generate(w)
+    K = t["K"].float()
+    # sink keys (positions 0..3) carry the large shared direction: norm about sqrt(1 + 9) x background
+    n_sink = K[:, :4].norm(dim=-1).mean()
+    n_bg = K[:, 100:].norm(dim=-1).mean()
+    assert n_sink > 2.5 * n_bg
+    # AR(1) with coefficient 0.8 along t
+    x = K[:, 100:-1].flatten()
+    y = K[:, 101:].flatten()
+    rho = torch.corrcoef(torch.stack([x, y]))[0, 1].item()
+    assert abs(rho - 0.8) < 0.02
+    assert abs(n_bg.item() / (0.5 * math.sqrt(w.d)) - 1.0) < 0.05
+
+
+def test_video_frames_correlated():
+    w = workloads.get(4, L=4096)
+    K = workloads.generate(w)["K"].float()
+    same = torch.nn.functional.cosine_similarity(K[0, 10], K[0, 900], dim=0)
+    assert same > 0.6
