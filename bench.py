@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the RRAttention sparse prefill layer (estimate + select + sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+
+One step = one full layer of the named workload (default: the Llama-3-8B-shaped layer at
+L = 131072, 32/8 heads, d = 128, S = 16, B = 128, tau = 0.9) on seeded synthetic bf16 inputs.
+Prints one JSON line.  ``value`` is effective TFLOP/s: dense-causal attention FLOPs
+4*d*H*L(L+1)/2 per layer, times the layers all ranks processed, divided by the max-over-ranks
+device time.  Under torchrun each rank runs its own layer (independent problems, weak
+scaling, no data-path collective).  ``--impl reference`` times the CPU oracle on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "ms/layer sparse prefill (estimate+select+attn) at 128K; effective TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def dense_causal_flops(w) -> float:
+    return 4.0 * w.d * w.H * w.L * (w.L + 1) / 2.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        loaded = [x for x in sm if x >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, t, n_rows: int, rng_seed: int = 0):
+    """Time the oracle on one query head's estimate + select and n_rows prefill rows of that
+    head; extrapolate linearly to the whole layer.  Returns (layer_seconds, info)."""
+    import oracle
+
+    h = 0
+    t0 = time.perf_counter()
+    A = oracle.estimate(t["Q"], t["K"], w.S, w.B, heads=(h, h + 1))
+    t1 = time.perf_counter()
+    rp, ci = oracle.select(A[h:h + 1], w.tau, True)
+    t2 = time.perf_counter()
+    rng = np.random.default_rng(rng_seed)
+    qs = np.sort(rng.choice(w.L, n_rows, replace=False))
+    # the head-0 CSR is rows 0..Nb-1 of a one-head CSR: run the oracle on head 0 alone
+    rows = [(0, int(q)) for q in qs]
+    oracle.prefill_rows(t["Q"][h:h + 1], t["K"][:1], t["V"][:1], w.B, rp, ci, rows)
+    t3 = time.perf_counter()
+    est, sel, pre = t1 - t0, t2 - t1, t3 - t2
+    # prefill cost grows with the number of attended keys: scale the sampled rows' time by
+    # (keys attended by all rows of the head) / (keys attended by the sampled rows)
+    B = w.B
+    n_off = np.zeros(w.Nb, np.int64)
+    has_diag = np.zeros(w.Nb, bool)
+    for I in range(w.Nb):
+        sel_I = ci[rp[I]:rp[I + 1]]
+        has_diag[I] = bool((sel_I == I).any())
+        n_off[I] = len(sel_I) - int(has_diag[I])
+    keys_all = float((n_off * B * B).sum() + has_diag.sum() * B * (B + 1) / 2)
+    Iq = qs // B
+    keys_sample = float((n_off[Iq] * B + has_diag[Iq] * (qs - Iq * B + 1)).sum())
+    layer = w.H * (est + sel + pre * keys_all / max(keys_sample, 1.0))
+    info = {"estimate_s_per_head": est, "select_s_per_head": sel, "prefill_s_sample": pre,
+            "rows": n_rows, "seconds_measured": t3 - t0}
+    return layer, info
+
+
+# ---------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    w = workloads.get(args.workload)
+    if args.L:
+        w = w.with_(L=args.L)
+    t = workloads.generate(w)
+    times = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        layer_s, info = oracle_sample(w, t, n_rows=args.ref_rows, rng_seed=i)
+        if i >= args.warmup:
+            times.append(layer_s)
+    ms = 1e3 * statistics.median(times)
+    val = dense_causal_flops(w) / (ms * 1e-3) / 1e12
+    sample = (f"per step: oracle estimate+select of query head 0 (all {w.Nb} query blocks) and "
+              f"{args.ref_rows} prefill rows of head 0; extrapolated linearly to {w.H} heads and "
+              f"{w.L} rows (prefill scaled by attended keys)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, world),
+        "cpu_baseline": {"kind": "oracle", "value": val, "unit": "TFLOP/s",
+                         "cores": oracle.threads(), "sample": sample, "last_step": info},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, world):
+    return {"workload": w.name, "H": w.H, "Hkv": w.Hkv, "L": w.L, "d": w.d, "S": w.S, "B": w.B,
+            "tau": w.tau, "recipe": w.recipe, "global_batch": world, "seq_len": w.L,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (Q+K+V %.2f GB > 126 MB); no flush" %
+                  (2 * w.L * w.d * (w.H + 2 * w.Hkv) / 1e9)}
+
+
+# ---------------------------------------------------------------------------- our arm
+def selected_flops(rp, ci, H, Nb, B, d):
+    rows = np.repeat(np.arange(H * Nb) % Nb, np.diff(rp))
+    diag = int((ci == rows).sum())
+    off = len(ci) - diag
+    return 4.0 * d * (off * B * B + diag * B * (B + 1) / 2.0), diag, off
+
+
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    import long_context_prefill_estimate_b200 as rr
+
+    rr.lib()  # fail loudly if the CUDA library is missing
+    w = workloads.get(args.workload)
+    if args.L:
+        w = w.with_(L=args.L)
+    host = workloads.generate(w, seed=rank)
+    d = {k: v.to(dev) for k, v in host.items()}
+    Q, K, V = d["Q"], d["K"], d["V"]
+    ws = rr.Workspace(w.H, w.Hkv, w.L, w.d, w.S, w.B, device=dev)
+    O = torch.empty_like(Q)
+    st = torch.cuda.current_stream(dev)
+
+    def step(ev=None, tau=None):
+        if ev:
+            ev[0].record(st)
+        rr.estimate(Q, K, w.S, w.B, out=ws.block_scores, workspace=ws.est)
+        if ev:
+            ev[1].record(st)
+        rr.select(ws.block_scores, w.tau if tau is None else tau, True, row_ptr=ws.row_ptr,
+                  col_idx=ws.col_idx, nnz=ws.nnz, workspace=ws.sel)
+        if ev:
+            ev[2].record(st)
+        rr.sparse_prefill(Q, K, V, ws.row_ptr, ws.col_idx, w.B, out=O)
+        if ev:
+            ev[3].record(st)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clk = ClockSampler(dev.index if dev.index is not None else 0)
+    clk.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(st)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = clk.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / args.steps
+    stage = {k: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+             for k, (a, b) in {"estimate_ms": (0, 1), "select_ms": (1, 2),
+                               "prefill_ms": (2, 3)}.items()}
+    rp = ws.row_ptr.cpu().numpy()
+    nnz = int(rp[-1])
+    ci = ws.col_idx[:nnz].cpu().numpy()
+    sel_flops, n_diag, n_off = selected_flops(rp, ci, w.H, w.Nb, w.B, w.d)
+    causal_blocks = w.H * w.Nb * (w.Nb + 1) // 2
+    dense = dense_causal_flops(w)
+    peaks, peak_kind = load_peaks()
+    prefill_tflops = sel_flops / (stage["prefill_ms"] * 1e-3) / 1e12
+    est_bytes = (2 * w.Hkv * w.L * w.d              # K read
+                 + 2 * w.H * w.Ns * w.d             # sampled Q rows
+                 + 4 * w.Hkv * w.Ns * w.d * 2       # pooled keys written + read
+                 + 4 * w.H * w.Nb * w.Nb)           # block scores written
+    sel_bytes = 4 * w.H * w.Nb * w.Nb + 4 * (w.H * w.Nb + 1) + 4 * nnz
+    line = {
+        "metric": METRIC,
+        "value": world * dense / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "ms_per_layer": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded generator, no datasets or weights)",
+        "config": config_dict(w, world),
+        "stages": {**stage,
+                   "estimate_gbs": est_bytes / (stage["estimate_ms"] * 1e-3) / 1e9,
+                   "select_gbs": sel_bytes / (stage["select_ms"] * 1e-3) / 1e9,
+                   "prefill_tflops_selected": prefill_tflops},
+        "density": nnz / causal_blocks,
+        "selected_blocks": nnz, "diag_blocks": n_diag,
+        "roofline": {"kernel": "sparse prefill", "bound": "tensor", "achieved": prefill_tflops,
+                     "peak": peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                     "unit": "TFLOP/s",
+                     "frac": prefill_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                     "frac_of_burst": prefill_tflops / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_kind} bf16 (sustained)",
+                     "flops_per_launch": sel_flops, "traffic": None},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks,
+    }
+    # ---- extra measurements (outside the timed region)
+    if rank == 0 and not args.quick:
+        line["tau_sweep"] = tau_sweep(w, step, st, ws, torch)
+        line["dense_reference"] = dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_step)
+    line["e2e"] = e2e(w, host, rr, torch, dev, args)
+    if rank == 0 and not args.no_cpu_baseline:
+        layer_s, info = oracle_sample(w, host, n_rows=args.cpu_rows)
+        import oracle
+
+        line["cpu_baseline"] = {
+            "value": dense / layer_s / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": (f"oracle estimate+select of query head 0 (all {w.Nb} query blocks) and "
+                       f"{args.cpu_rows} prefill rows of head 0, extrapolated linearly to the "
+                       f"layer ({layer_s:.1f} s/layer); measured {info['seconds_measured']:.1f} s"),
+        }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def tau_sweep(w, step, st, ws, torch):
+    out = {}
+    for tau in (0.8, 0.9, 0.95):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        step(tau=tau)
+        torch.cuda.synchronize()
+        step(ev, tau=tau)
+        torch.cuda.synchronize()
+        nnz = int(ws.row_ptr[-1].item())
+        out[str(tau)] = {"density": nnz / (w.H * w.Nb * (w.Nb + 1) // 2),
+                         "ms": ev[0].elapsed_time(ev[3]),
+                         "prefill_ms": ev[2].elapsed_time(ev[3])}
+    return out
+
+
+def dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_sparse):
+    """Dense causal attention on the same GPU: our kernel with every causal block, and torch
+    SDPA (flash/cuDNN library kernel) as context."""
+    res = {}
+    Nb = w.Nb
+    counts = np.tile(np.arange(1, Nb + 1), w.H)
+    rp = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(Q.device)
+    ci = torch.from_numpy(np.concatenate([np.arange(I + 1) for _ in range(w.H) for I in range(Nb)]
+                                         ).astype(np.int32)).to(Q.device)
+    O = torch.empty_like(Q)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rr.sparse_prefill(Q, K, V, rp, ci, w.B, out=O)
+    e0.record(st)
+    rr.sparse_prefill(Q, K, V, rp, ci, w.B, out=O)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    res["ours_tau1_ms"] = ms
+    res["ours_tau1_tflops"] = dense_causal_flops(w) / (ms * 1e-3) / 1e12
+    res["speedup_vs_ours_dense"] = ms / ms_sparse
+    try:
+        G = w.H // w.Hkv
+        q = Q.unsqueeze(0)
+        k = K.unsqueeze(0)
+        v = V.unsqueeze(0)
+        torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+        e0.record(st)
+        torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+        e1.record(st)
+        torch.cuda.synchronize()
+        ms2 = e0.elapsed_time(e1)
+        res["sdpa_ms"] = ms2
+        res["sdpa_tflops"] = dense_causal_flops(w) / (ms2 * 1e-3) / 1e12
+        res["speedup_vs_sdpa"] = ms2 / ms_sparse
+        del G
+    except Exception as exc:  # library kernel unavailable for this shape
+        res["sdpa_error"] = str(exc)[:200]
+    return res
+
+
+def e2e(w, host, rr, torch, dev, args):
+    """Same layer through the public API from pinned host buffers: H2D of Q/K/V, the three
+    stages, D2H of O, every step inside the timed region."""
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    out = torch.empty(pinned["Q"].shape, dtype=torch.bfloat16, pin_memory=True)
+    ws = rr.Workspace(w.H, w.Hkv, w.L, w.d, w.S, w.B, device=dev)
+    st = torch.cuda.current_stream(dev)
+    for _ in range(max(1, min(args.warmup, 2))):
+        rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, ws=ws, out=out)
+    n = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(n):
+        rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, ws=ws, out=out)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    return {"value": world * dense_causal_flops(w) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, help="index into workloads.WORKLOADS")
+    ap.add_argument("--L", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--quick", action="store_true", help="skip the tau sweep and dense comparison")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,234 @@
+"""RRAttention sparse prefill on NVIDIA B200 -- Python binding of librrattn.so.
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  There is no CPU fallback: if
+the library is missing, or a tensor is not on a CUDA device, calls raise.
+
+    estimate(Q, K, S, B)              -> block_scores [H][L/B][L/B] float32
+    select(block_scores, tau)         -> (row_ptr int32 [H*Nb+1], col_idx int32, nnz)
+    sparse_prefill(Q, K, V, row_ptr, col_idx, B) -> O [H][L][d] bf16
+    prefill(Q, K, V, S, B, tau)       -> O (the three stages back to back)
+
+Shapes: Q [H][L][d], K and V [Hkv][L][d], contiguous bf16 on one CUDA device.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
+           "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
+           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "librrattn.so")
+
+STRATEGIES = {"head": 0, "none": 1, "layer": 2, "hybrid": 3}
+
+EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_workspace_bytes",
+                    "rr_select", "rr_select_workspace_bytes", "rr_sparse_prefill",
+                    "rr_validate_csr", "rr_status_string", "rr_last_error", "rr_version")
+
+
+class RRAttnError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {_STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+_STATUS = {0: "RR_OK", 1: "RR_ERR_INVALID_ARG", 2: "RR_ERR_UNSUPPORTED", 3: "RR_ERR_CUDA",
+           4: "RR_ERR_WORKSPACE"}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded librrattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RRAttnError("load", -1, f"{library_path} is missing: build it with "
+                          "`python -m long_context_prefill_estimate_b200.build`")
+    L = ctypes.CDLL(library_path)
+    P, I, Z, F, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_double
+    I64 = ctypes.c_int64
+    L.rr_estimate_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    L.rr_estimate_workspace_bytes.restype = Z
+    L.rr_estimate.argtypes = [P, P, I, I, I, I, I, I, P, P, Z, P]
+    L.rr_estimate.restype = I
+    L.rr_estimate_strategy.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P, Z, P]
+    L.rr_estimate_strategy.restype = I
+    L.rr_select_workspace_bytes.argtypes = [I, I]
+    L.rr_select_workspace_bytes.restype = Z
+    L.rr_select.argtypes = [P, I, I, D, I, P, P, I64, P, P, Z, P]
+    L.rr_select.restype = I
+    L.rr_sparse_prefill.argtypes = [P, P, P, I, I, I, I, I, P, P, F, P, P]
+    L.rr_sparse_prefill.restype = I
+    L.rr_validate_csr.argtypes = [P, P, I, I, I64, P, P]
+    L.rr_validate_csr.restype = I
+    L.rr_status_string.argtypes = [I]
+    L.rr_status_string.restype = ctypes.c_char_p
+    L.rr_last_error.argtypes = []
+    L.rr_last_error.restype = ctypes.c_char_p
+    L.rr_version.restype = I
+    _lib = L
+    return L
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise RRAttnError(fn, code, lib().rr_last_error().decode(errors="replace"))
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype: torch.dtype):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise RRAttnError(name, 1, "tensors must live on a CUDA device (no CPU path exists)")
+    if t.dtype != dtype:
+        raise RRAttnError(name, 1, f"expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise RRAttnError(name, 1, "tensors must be contiguous")
+
+
+def estimate_workspace_bytes(H: int, Hkv: int, L: int, d: int, S: int, B: int) -> int:
+    return int(lib().rr_estimate_workspace_bytes(H, Hkv, L, d, S, B))
+
+
+def select_workspace_bytes(H: int, Nb: int) -> int:
+    return int(lib().rr_select_workspace_bytes(H, Nb))
+
+
+class Workspace:
+    """Reusable device buffers for one layer shape (avoids per-call allocation)."""
+
+    def __init__(self, H: int, Hkv: int, L: int, d: int, S: int, B: int, device="cuda"):
+        self.shape = (H, Hkv, L, d, S, B)
+        Nb = L // B
+        dev = torch.device(device)
+        self.est = torch.empty(max(estimate_workspace_bytes(H, Hkv, L, d, S, B), 16),
+                               dtype=torch.uint8, device=dev)
+        self.sel = torch.empty(max(select_workspace_bytes(H, Nb), 16), dtype=torch.uint8, device=dev)
+        self.block_scores = torch.empty((H, Nb, Nb), dtype=torch.float32, device=dev)
+        self.row_ptr = torch.empty(H * Nb + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(max(H * Nb * (Nb + 1) // 2, 1), dtype=torch.int32, device=dev)
+        self.nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+
+
+def estimate(Q: torch.Tensor, K: torch.Tensor, S: int, B: int, strategy: str = "head",
+             layer: int = 0, out: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block importance [H][L/B][L/B] (float32) from round-robin sampled queries."""
+    _need_cuda("rr_estimate", Q, torch.bfloat16)
+    _need_cuda("rr_estimate", K, torch.bfloat16)
+    H, L, d = Q.shape
+    Hkv = K.shape[0]
+    if K.shape != (Hkv, L, d):
+        raise RRAttnError("rr_estimate", 1, f"K shape {tuple(K.shape)} does not match Q {tuple(Q.shape)}")
+    Nb = L // B if B > 0 else 0
+    if out is None:
+        out = torch.empty((H, Nb, Nb), dtype=torch.float32, device=Q.device)
+    need = estimate_workspace_bytes(H, Hkv, L, d, S, B)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=Q.device)
+    _check("rr_estimate", lib().rr_estimate_strategy(
+        _ptr(Q), _ptr(K), H, Hkv, L, d, S, B, STRATEGIES[strategy], layer, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(Q.device)))
+    return out
+
+
+def select(block_scores: torch.Tensor, tau: float, protect_last: bool = True,
+           row_ptr: Optional[torch.Tensor] = None, col_idx: Optional[torch.Tensor] = None,
+           nnz: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None
+           ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Top-tau CSR block lists.  col_idx has worst-case capacity; nnz (device int64) and
+    row_ptr[-1] give the used length."""
+    _need_cuda("rr_select", block_scores, torch.float32)
+    H, Nb, Nb2 = block_scores.shape
+    if Nb != Nb2:
+        raise RRAttnError("rr_select", 1, "block_scores must be [H][Nb][Nb]")
+    dev = block_scores.device
+    cap = max(H * Nb * (Nb + 1) // 2, 1)
+    if row_ptr is None:
+        row_ptr = torch.empty(H * Nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(cap, dtype=torch.int32, device=dev)
+    if nnz is None:
+        nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(select_workspace_bytes(H, Nb), 16), dtype=torch.uint8, device=dev)
+    _check("rr_select", lib().rr_select(
+        _ptr(block_scores), H, Nb, float(tau), int(bool(protect_last)), _ptr(row_ptr),
+        _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(workspace), workspace.numel(),
+        _stream(dev)))
+    return row_ptr, col_idx, nnz
+
+
+def sparse_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: torch.Tensor,
+                   col_idx: torch.Tensor, B: int, scale: Optional[float] = None,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Causal block-sparse attention over the CSR-selected blocks -> O [H][L][d] bf16."""
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _need_cuda("rr_sparse_prefill", t, torch.bfloat16)
+    _need_cuda("rr_sparse_prefill", row_ptr, torch.int32)
+    _need_cuda("rr_sparse_prefill", col_idx, torch.int32)
+    H, L, d = Q.shape
+    Hkv = K.shape[0]
+    if K.shape != (Hkv, L, d) or V.shape != K.shape:
+        raise RRAttnError("rr_sparse_prefill", 1, "K/V shapes do not match Q")
+    if out is None:
+        out = torch.empty_like(Q)
+    _check("rr_sparse_prefill", lib().rr_sparse_prefill(
+        _ptr(Q), _ptr(K), _ptr(V), H, Hkv, L, d, B, _ptr(row_ptr), _ptr(col_idx),
+        float(scale) if scale else 0.0, _ptr(out), _stream(Q.device)))
+    return out
+
+
+def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, tau: float,
+            protect_last: bool = True, strategy: str = "head", layer: int = 0,
+            scale: Optional[float] = None, ws: Optional[Workspace] = None,
+            out: Optional[torch.Tensor] = None, return_intermediates: bool = False):
+    """One attention layer's sparse prefill: estimate -> select -> sparse attention.
+
+    Host (CPU) tensors are accepted: they are copied to the current CUDA device and the
+    output is copied back (pinned host memory makes those copies asynchronous)."""
+    host = not Q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        Q, K, V = (t.to(dev, non_blocking=True) for t in (Q, K, V))
+    H, L, d = Q.shape
+    Hkv = K.shape[0]
+    if ws is None:
+        ws = Workspace(H, Hkv, L, d, S, B, device=Q.device)
+    estimate(Q, K, S, B, strategy=strategy, layer=layer, out=ws.block_scores, workspace=ws.est)
+    select(ws.block_scores, tau, protect_last, row_ptr=ws.row_ptr, col_idx=ws.col_idx,
+           nnz=ws.nnz, workspace=ws.sel)
+    O = sparse_prefill(Q, K, V, ws.row_ptr, ws.col_idx, B, scale=scale,
+                       out=None if host else out)
+    if host:
+        dst = out if out is not None else torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+        dst.copy_(O, non_blocking=True)
+        torch.cuda.current_stream(O.device).synchronize()
+        O = dst
+    if return_intermediates:
+        return O, ws
+    return O
+
+
+def validate_csr(row_ptr: torch.Tensor, col_idx: torch.Tensor, H: int, Nb: int) -> int:
+    """Number of malformed CSR rows (checked on the device; synchronises to read it)."""
+    bad = torch.zeros(1, dtype=torch.int32, device=row_ptr.device)
+    _check("rr_validate_csr", lib().rr_validate_csr(
+        _ptr(row_ptr), _ptr(col_idx), H, Nb, col_idx.numel(), _ptr(bad), _stream(row_ptr.device)))
+    return int(bad.item())

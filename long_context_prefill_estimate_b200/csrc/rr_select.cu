@@ -1,0 +1,269 @@
+// Adaptive Top-tau block selection of RRAttention ("RRAttention: Dynamic Block Sparse
+// Attention via Per-Head Round-Robin Shifts for Long-Context Inference", Sec. 1 contribution
+// (iii), Sec. 3.3 heading; the rule as the XAttention card states it: the smallest set of
+// blocks whose cumulative score reaches tau) with last-query-block protection (Sec. 4.3).
+//
+//   select_rows_kernel  one CTA per (head, query block) row: bitonic sort of the row's
+//                       causal scores on the key (score desc, J asc), float64 inclusive scan,
+//                       k* = 1 + #{k : cum_k < tau*T}, selected blocks as a bitmap.
+//   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr, nnz.
+//   emit_csr_kernel     one warp per row: bitmap -> ascending block indices in col_idx.
+//   validate_csr_kernel debug check of a CSR, counts bad rows, never traps.
+#include "rr_common.cuh"
+
+namespace rr {
+
+namespace {
+
+constexpr int kSelThreads = 256;
+
+__device__ __forceinline__ uint64_t sort_key(float a, int J) {
+    uint32_t bits = __float_as_uint(a);
+    if (a == 0.f) bits = 0;  // -0 sorts as +0
+    return ((uint64_t)(~bits) << 32) | (uint32_t)J;
+}
+
+__device__ __forceinline__ double key_value(uint64_t k) {
+    return (double)__uint_as_float(~(uint32_t)(k >> 32));
+}
+
+// Block-wide exclusive scan of one value per thread (double), returns the exclusive prefix
+// and writes the block total to *total.
+__device__ double block_exclusive_scan(double v, double *warp_tot, double *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    double x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        double t = lane < nw ? warp_tot[lane] : 0.0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < nw) warp_tot[lane] = t;  // inclusive per warp
+        if (lane == nw - 1) *total = t;
+    }
+    __syncthreads();
+    const double before = warp ? warp_tot[warp - 1] : 0.0;
+    return before + x - v;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    select_rows_kernel(const float *__restrict__ A, int Nb, double tau, int protect_last, int P,
+                       int W, int *__restrict__ counts, uint32_t *__restrict__ bitmap) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);
+    uint32_t *bm = reinterpret_cast<uint32_t *>(smem_raw + (size_t)P * 8);
+    __shared__ double warp_tot[32];
+    __shared__ double s_total;
+    __shared__ int s_below;
+
+    const long row = blockIdx.x;
+    const int I = (int)(row % Nb), n = I + 1, tid = threadIdx.x;
+    uint32_t *out_bm = bitmap + row * W;
+    const bool keep_all = (tau >= 1.0) || (protect_last && I == Nb - 1);
+    if (keep_all) {
+        for (int w = tid; w < W; w += kSelThreads) {
+            const int lo = w * 32;
+            uint32_t m = 0;
+            if (n >= lo + 32) m = 0xffffffffu;
+            else if (n > lo) m = (1u << (n - lo)) - 1u;
+            out_bm[w] = m;
+        }
+        if (tid == 0) counts[row] = n;
+        return;
+    }
+    const float *a = A + row * (long)Nb;
+    for (int k = tid; k < P; k += kSelThreads) keys[k] = (k < n) ? sort_key(__ldg(a + k), k) : ~0ull;
+    for (int w = tid; w < W; w += kSelThreads) bm[w] = 0;
+    if (tid == 0) s_below = 0;
+    __syncthreads();
+    // bitonic sort, ascending keys
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = tid; t < P / 2; t += kSelThreads) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = ((lo & size) == 0);
+                const uint64_t x = keys[lo], y = keys[hi];
+                if ((x > y) == up) {
+                    keys[lo] = y;
+                    keys[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    // each thread owns a contiguous chunk of the sorted order
+    const int per = (P + kSelThreads - 1) / kSelThreads;
+    const int k0 = tid * per, k1 = min(k0 + per, n);
+    double local = 0.0;
+    for (int k = k0; k < k1; ++k) local += key_value(keys[k]);
+    const double base = block_exclusive_scan(local, warp_tot, &s_total);
+    const double T = s_total;  // all n values summed (pads excluded)
+    const double thr = tau * T;
+    int below = 0;
+    double cum = base;
+    for (int k = k0; k < k1; ++k) {
+        cum += key_value(keys[k]);
+        below += (cum < thr);
+    }
+    if (below) atomicAdd(&s_below, below);
+    __syncthreads();
+    const int kstar = min(s_below + 1, n);
+    for (int k = tid; k < kstar; k += kSelThreads) {
+        const int J = (int)(keys[k] & 0xffffffffu);
+        atomicOr(&bm[J >> 5], 1u << (J & 31));
+    }
+    __syncthreads();
+    for (int w = tid; w < W; w += kSelThreads) out_bm[w] = bm[w];
+    if (tid == 0) counts[row] = kstar;
+}
+
+__global__ void __launch_bounds__(1024)
+    scan_counts_kernel(const int *__restrict__ counts, long nrows, int32_t *__restrict__ row_ptr,
+                       int64_t *__restrict__ nnz_out) {
+    __shared__ long warp_tot[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long per = (nrows + 1023) / 1024;
+    const long r0 = tid * per, r1 = min(r0 + per, nrows);
+    long local = 0;
+    for (long r = r0; r < r1; ++r) local += counts[r];
+    long x = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        long t = warp_tot[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            const long y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        warp_tot[lane] = t;
+    }
+    __syncthreads();
+    long at = (warp ? warp_tot[warp - 1] : 0) + x - local;
+    for (long r = r0; r < r1; ++r) {
+        row_ptr[r] = (int32_t)at;
+        at += counts[r];
+    }
+    if (tid == 1023) {
+        row_ptr[nrows] = (int32_t)warp_tot[31];
+        if (nnz_out) *nnz_out = warp_tot[31];
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    emit_csr_kernel(const uint32_t *__restrict__ bitmap, const int32_t *__restrict__ row_ptr,
+                    long nrows, int W, int32_t *__restrict__ col_idx) {
+    const long row = blockIdx.x * 8L + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= nrows) return;
+    const uint32_t *bm = bitmap + row * W;
+    int at = row_ptr[row];
+    for (int w0 = 0; w0 < W; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t m = (w < W) ? bm[w] : 0u;
+        const int c = __popc(m);
+        int x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        int pos = at + x - c;
+        uint32_t mm = m;
+        while (mm) {
+            const int b = __ffs(mm) - 1;
+            col_idx[pos++] = w * 32 + b;
+            mm &= mm - 1;
+        }
+        at += __shfl_sync(0xffffffffu, x, 31);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    validate_csr_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                        int Nb, long nrows, long nnz_cap, int32_t *__restrict__ bad) {
+    for (long row = blockIdx.x * (long)blockDim.x + threadIdx.x; row < nrows;
+         row += (long)gridDim.x * blockDim.x) {
+        const int I = (int)(row % Nb);
+        const long b = row_ptr[row], e = row_ptr[row + 1];
+        bool ok = (row != 0 || b == 0) && b >= 0 && e > b && e <= nnz_cap;
+        if (ok) {
+            int prev = -1;
+            for (long c = b; c < e && ok; ++c) {
+                const int J = col_idx[c];
+                ok = (J > prev) && (J <= I);
+                prev = J;
+            }
+        }
+        if (!ok) atomicAdd(bad, 1);
+    }
+}
+
+}  // namespace
+
+static int pow2_at_least(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+size_t select_workspace_bytes(int H, int Nb) {
+    if (H <= 0 || Nb <= 0) return 0;
+    const size_t nrows = (size_t)H * Nb, W = (Nb + 31) / 32;
+    return align_up(nrows * 4, 256) + nrows * W * 4;
+}
+
+size_t select_smem_bytes(int Nb) {
+    const int P = pow2_at_least(Nb < 2 ? 2 : Nb);
+    return (size_t)P * 8 + (size_t)((P + 31) / 32) * 4;
+}
+
+rr_status_t launch_select(const float *A, int H, int Nb, double tau, int protect_last,
+                          int32_t *row_ptr, int32_t *col_idx, int64_t *nnz_out, void *ws,
+                          cudaStream_t st) {
+    const long nrows = (long)H * Nb;
+    const int W = (Nb + 31) / 32;
+    const int P = pow2_at_least(Nb < 2 ? 2 : Nb);
+    int *counts = static_cast<int *>(ws);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + align_up(nrows * 4, 256));
+    const size_t smem = select_smem_bytes(Nb);
+    cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return set_error(RR_ERR_CUDA, "rr_select: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    select_rows_kernel<<<(unsigned)nrows, kSelThreads, smem, st>>>(A, Nb, tau, protect_last, P, W,
+                                                                   counts, bitmap);
+    rr_status_t s = check_launch("rr_select: select_rows_kernel");
+    if (s != RR_OK) return s;
+    scan_counts_kernel<<<1, 1024, 0, st>>>(counts, nrows, row_ptr, nnz_out);
+    s = check_launch("rr_select: scan_counts_kernel");
+    if (s != RR_OK) return s;
+    emit_csr_kernel<<<(unsigned)((nrows + 7) / 8), 256, 0, st>>>(bitmap, row_ptr, nrows, W, col_idx);
+    return check_launch("rr_select: emit_csr_kernel");
+}
+
+rr_status_t launch_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int H, int Nb,
+                                int64_t nnz_cap, int32_t *bad, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(bad, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess)
+        return set_error(RR_ERR_CUDA, "rr_validate_csr: memset: %s", cudaGetErrorString(e));
+    const long nrows = (long)H * Nb;
+    const long want = (nrows + 255) / 256;
+    validate_csr_kernel<<<(unsigned)(want < 4096 ? want : 4096), 256, 0, st>>>(row_ptr, col_idx, Nb,
+                                                                               nrows, nnz_cap, bad);
+    return check_launch("rr_validate_csr");
+}
+
+}  // namespace rr

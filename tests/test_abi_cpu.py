@@ -1,0 +1,110 @@
+"""C-ABI library: loads, exports every symbol the header declares, validates on the host.
+
+No compute call is made here: every call below is rejected by host-side validation before
+any CUDA API is touched, so this runs on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_prefill_estimate_b200 as rr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rr_attn.h")
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 4
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rr_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_prefill_estimate_b200 import build
+
+    build.build()
+    return rr.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert set(names) >= {"rr_estimate", "rr_select", "rr_sparse_prefill"}
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in rr_attn.h but not exported"
+    assert set(rr.EXPORTED_SYMBOLS) == set(names)
+
+
+def test_version_and_status_strings(L):
+    assert L.rr_version() >= 100
+    assert L.rr_status_string(0) == b"RR_OK"
+    assert L.rr_status_string(4) == b"RR_ERR_WORKSPACE"
+    assert L.rr_status_string(99) == b"RR_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(L):
+    assert rr.estimate_workspace_bytes(32, 8, 131072, 128, 16, 128) == 8 * 8192 * 128 * 4
+    assert rr.estimate_workspace_bytes(32, 8, 0, 128, 16, 128) == 0
+    assert rr.select_workspace_bytes(32, 1024) >= 32 * 1024 * 4 + 32 * 1024 * 32 * 4
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+def _est(L, H=4, Hkv=2, Len=256, d=64, S=8, B=64, strategy=0, layer=0, q=FAKE, k=FAKE, out=FAKE,
+         ws=FAKE, wsb=1 << 30):
+    return L.rr_estimate_strategy(q, k, H, Hkv, Len, d, S, B, strategy, layer, out, ws, wsb, None)
+
+
+def test_estimate_rejections(L):
+    assert _est(L, H=3, Hkv=2) == INVALID
+    assert _est(L, d=96) == UNSUPPORTED
+    assert _est(L, B=32) == UNSUPPORTED
+    assert _est(L, Len=200) == UNSUPPORTED
+    assert _est(L, S=3) == INVALID
+    assert _est(L, S=16) == UNSUPPORTED        # B/S = 4 is not a multiple of 8
+    assert _est(L, strategy=7) == INVALID
+    assert _est(L, q=0) == INVALID
+    assert _est(L, k=FAKE + 4) == INVALID      # misaligned
+    assert _est(L, ws=0) == WORKSPACE
+    assert _est(L, wsb=16) == WORKSPACE
+    assert b"workspace" in L.rr_last_error()
+    assert _est(L, Len=0, q=0, k=0, out=0, ws=0) == 0   # empty problem: accepted, no launch
+
+
+def test_select_rejections(L):
+    P = FAKE
+    ok_cap = 2 * 4 * 5 // 2
+    assert L.rr_select(P, 2, 4, 0.0, 1, P, P, ok_cap, None, P, 1 << 20, None) == INVALID
+    assert L.rr_select(P, 2, 4, 1.5, 1, P, P, ok_cap, None, P, 1 << 20, None) == INVALID
+    assert L.rr_select(P, 2, 4, float("nan"), 1, P, P, ok_cap, None, P, 1 << 20, None) == INVALID
+    assert L.rr_select(P, 2, 4, 0.9, 1, P, P, ok_cap - 1, None, P, 1 << 20, None) == INVALID
+    assert b"col_capacity" in L.rr_last_error()
+    assert L.rr_select(P, 2, 4, 0.9, 1, P, P, ok_cap, None, P, 8, None) == WORKSPACE
+    assert L.rr_select(P, 2, 4, 0.9, 1, P, P, ok_cap, P + 4, P, 1 << 20, None) == INVALID
+    assert L.rr_select(0, 2, 0, 0.9, 1, 0, 0, 0, None, 0, 0, None) == 0  # empty
+
+
+def test_prefill_rejections(L):
+    P = FAKE
+    f = L.rr_sparse_prefill
+    assert f(P, P, P, 4, 3, 256, 64, 64, P, P, 0.0, P, None) == INVALID
+    assert f(P, P, P, 4, 2, 256, 80, 64, P, P, 0.0, P, None) == UNSUPPORTED
+    assert f(P, P, P, 4, 2, 250, 64, 64, P, P, 0.0, P, None) == UNSUPPORTED
+    assert f(P, P, P, 4, 2, 256, 64, 64, 0, P, 0.0, P, None) == INVALID
+    assert f(P, P, P, 4, 2, 256, 64, 64, P, P, float("inf"), P, None) == INVALID
+    assert f(0, 0, 0, 4, 2, 0, 64, 64, 0, 0, 0.0, 0, None) == 0
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+
+    Q = torch.zeros(2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(rr.RRAttnError, match="CUDA device"):
+        rr.estimate(Q, Q, 8, 64)
+    with pytest.raises(rr.RRAttnError, match="CUDA device"):
+        rr.sparse_prefill(Q, Q, Q, torch.zeros(3, dtype=torch.int32), torch.zeros(3, dtype=torch.int32), 64)
