@@ -108,6 +108,25 @@ rr_status_t rr_select(const float *block_scores, int H, int Nb, double tau, int 
                       rr_stream_t stream);
 
 /*
+ * rr_select_noalloc -- rr_select without a caller-provided workspace.  The paper has no
+ * counterpart to this call: it exists for callers that cannot allocate device memory (a
+ * plugin whose host application owns all device memory and offers no allocation hook, or a
+ * latency-critical path that must not call cudaMalloc/cudaFree).  Same arguments, results
+ * and validation as rr_select, minus workspace/workspace_bytes; the library allocates
+ * nothing and calls no allocating routine.
+ *
+ * Scratch: a fixed 8 MiB array compiled into the library (held by every GPU that loads it
+ * until the process exits).  Sizes with rr_select_workspace_bytes(H, Nb) > 8 MiB are rejected
+ * with RR_ERR_UNSUPPORTED before any launch.  The first call on a device (with that device
+ * current) looks up the array's device address once; make it before any stream capture.
+ * All calls share the array: calls that overlap on the GPU (unordered streams or threads)
+ * race; each call writes every scratch word it reads, so no clearing is needed.
+ */
+rr_status_t rr_select_noalloc(const float *block_scores, int H, int Nb, double tau,
+                              int protect_last, int32_t *row_ptr, int32_t *col_idx,
+                              int64_t col_capacity, int64_t *nnz_out, rr_stream_t stream);
+
+/*
  * rr_sparse_prefill -- causal block-sparse attention over the selected blocks (Sec. 2.1
  * with the CSR as the block selection matrix).  For query row t of head h, in block
  * I = t / B, key k of KV head g(h) is attended iff k <= t and k / B is listed in row

@@ -30,7 +30,8 @@ library_path = os.path.join(_HERE, "librrattn.so")
 STRATEGIES = {"head": 0, "none": 1, "layer": 2, "hybrid": 3}
 
 EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_workspace_bytes",
-                    "rr_select", "rr_select_workspace_bytes", "rr_sparse_prefill",
+                    "rr_select", "rr_select_workspace_bytes", "rr_select_noalloc",
+                    "rr_sparse_prefill",
                     "rr_validate_csr", "rr_status_string", "rr_last_error", "rr_version")
 
 
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.rr_select_workspace_bytes.restype = Z
     L.rr_select.argtypes = [P, I, I, D, I, P, P, I64, P, P, Z, P]
     L.rr_select.restype = I
+    L.rr_select_noalloc.argtypes = [P, I, I, D, I, P, P, I64, P, P]
+    L.rr_select_noalloc.restype = I
     L.rr_sparse_prefill.argtypes = [P, P, P, I, I, I, I, I, P, P, F, P, P]
     L.rr_sparse_prefill.restype = I
     L.rr_validate_csr.argtypes = [P, P, I, I, I64, P, P]
