@@ -149,6 +149,14 @@ rr_status_t rr_sparse_prefill(const rr_bf16_t *Q, const rr_bf16_t *K, const rr_b
 rr_status_t rr_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int H, int Nb,
                             int64_t nnz_cap, int32_t *bad_rows, rr_stream_t stream);
 
+/*
+ * rr_device_errors -- error bits the kernels recorded on the current device instead of
+ * trapping: bit 0 producer, bit 1 MMA issuer, bit 2 softmax warps of rr_sparse_prefill gave
+ * up a wait after about one second.  *flags (host) receives the bits; reset != 0 clears them.
+ * Synchronous: waits for the device's preceding work.
+ */
+rr_status_t rr_device_errors(uint32_t *flags, int reset);
+
 /* Static text for a status code. */
 const char *rr_status_string(rr_status_t s);
 

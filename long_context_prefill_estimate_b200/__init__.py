@@ -22,7 +22,7 @@ import torch
 
 __all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
            "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
-           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS"]
+           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "librrattn.so")
@@ -32,7 +32,8 @@ STRATEGIES = {"head": 0, "none": 1, "layer": 2, "hybrid": 3}
 EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_workspace_bytes",
                     "rr_select", "rr_select_workspace_bytes", "rr_select_noalloc",
                     "rr_sparse_prefill",
-                    "rr_validate_csr", "rr_status_string", "rr_last_error", "rr_version")
+                    "rr_validate_csr", "rr_device_errors", "rr_status_string", "rr_last_error",
+                    "rr_version")
 
 
 class RRAttnError(RuntimeError):
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.rr_sparse_prefill.restype = I
     L.rr_validate_csr.argtypes = [P, P, I, I, I64, P, P]
     L.rr_validate_csr.restype = I
+    L.rr_device_errors.argtypes = [P, I]
+    L.rr_device_errors.restype = I
     L.rr_status_string.argtypes = [I]
     L.rr_status_string.restype = ctypes.c_char_p
     L.rr_last_error.argtypes = []
@@ -235,3 +238,10 @@ def validate_csr(row_ptr: torch.Tensor, col_idx: torch.Tensor, H: int, Nb: int) 
     _check("rr_validate_csr", lib().rr_validate_csr(
         _ptr(row_ptr), _ptr(col_idx), H, Nb, col_idx.numel(), _ptr(bad), _stream(row_ptr.device)))
     return int(bad.item())
+
+
+def device_errors(reset: bool = True) -> int:
+    """Error bits recorded by the kernels on the current device (0 = none); synchronises."""
+    v = ctypes.c_uint32(0)
+    _check("rr_device_errors", lib().rr_device_errors(ctypes.byref(v), int(reset)))
+    return int(v.value)

@@ -20,10 +20,10 @@ rr_status_t launch_select(const float *A, int H, int Nb, double tau, int protect
                           cudaStream_t st);
 rr_status_t launch_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int H, int Nb,
                                 int64_t nnz_cap, int32_t *bad, cudaStream_t st);
-rr_status_t launch_prefill_mma(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H,
-                               int Hkv, int L, int d, int B, const int32_t *row_ptr,
-                               const int32_t *col_idx, float scale, uint16_t *O,
-                               cudaStream_t st);
+rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H, int Hkv,
+                              int L, int d, int B, const int32_t *row_ptr, const int32_t *col_idx,
+                              float scale, uint16_t *O, cudaStream_t st);
+rr_status_t read_device_errors(unsigned *out, bool reset);
 
 static thread_local char g_last_error[512] = "";
 
@@ -96,6 +96,15 @@ const char *rr_status_string(rr_status_t s) {
 }
 
 const char *rr_last_error(void) { return g_last_error; }
+
+rr_status_t rr_device_errors(uint32_t *flags, int reset) {
+    g_last_error[0] = 0;
+    if (!flags) return set_error(RR_ERR_INVALID_ARG, "rr_device_errors: flags is NULL");
+    unsigned v = 0;
+    const rr_status_t s = read_device_errors(&v, reset != 0);
+    *flags = v;
+    return s;
+}
 
 size_t rr_estimate_workspace_bytes(int H, int Hkv, int L, int d, int S, int B) {
     (void)H;
@@ -190,8 +199,8 @@ rr_status_t rr_sparse_prefill(const rr_bf16_t *Q, const rr_bf16_t *K, const rr_b
     RR_TRY(check_ptr(fn, "row_ptr", row_ptr));
     RR_TRY(check_ptr(fn, "col_idx", col_idx));
     const float scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)d));
-    return launch_prefill_mma(Q, K, V, H, Hkv, L, d, B, row_ptr, col_idx, scale, O,
-                              static_cast<cudaStream_t>(stream));
+    return launch_prefill_tc(Q, K, V, H, Hkv, L, d, B, row_ptr, col_idx, scale, O,
+                             static_cast<cudaStream_t>(stream));
 }
 
 rr_status_t rr_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int H, int Nb,

@@ -1,0 +1,397 @@
+// Causal block-sparse attention over the selected blocks on the 5th-generation tensor cores
+// ("RRAttention: Dynamic Block Sparse Attention via Per-Head Round-Robin Shifts for
+// Long-Context Inference", Sec. 2.1 with the per-head CSR block lists as the block selection
+// matrix; Sec. 4.1: sparsity in prefill only).
+//
+// One CTA per (query head h, query block I): a 128-row query tile (for B = 64 the upper 64
+// rows are padding that is computed and never stored).  The CTA walks only the CSR entries
+// of row h*Nb + I.  Warp roles:
+//   warp 0      TMA producer: Q tile once, then K and V tiles of each selected block into a
+//               2-stage ring (128-byte swizzle, mbarrier transaction counts).
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM buffers, then
+//               O += P_j V_j into a TMEM accumulator; completion signalled by tcgen05.commit.
+//   warp 2      TMEM allocation / release.
+//   warps 4-7   softmax: one thread per query row (TMEM lane), online softmax in fp32 with a
+//               lazily rescaled running max (O is rescaled in TMEM only when the max grows by
+//               more than 2^8), P written to shared memory in the MMA operand layout, final
+//               normalisation and bf16 store.
+// K and V come from KV head h / (H/Hkv); the heads of a KV group run as adjacent CTAs so
+// their K/V tiles are served from L2.  Every wait is bounded (about one second of
+// %globaltimer); a timeout sets a device error bit and the CTA drains and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "rr_common.cuh"
+#include "rr_sm100.cuh"
+
+namespace rr {
+
+namespace {
+
+__device__ unsigned int g_device_errors;
+
+constexpr unsigned kErrTimeoutProducer = 1u, kErrTimeoutMma = 2u, kErrTimeoutSoftmax = 4u;
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of `parity` to complete, for at most ~1 s.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (sm100::mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 0 && globaltimer() - t0 > 1000000000ull) return false;
+    }
+}
+
+constexpr int kBM = 128;  // query rows per CTA
+constexpr int kNS = 2;    // K/V pipeline stages
+
+template <int D, int BN>
+struct TcCfg {
+    static constexpr int DC = D / 64;                       // 64-element (128-byte) column chunks
+    static constexpr uint32_t Q_BYTES = kBM * D * 2;
+    static constexpr uint32_t KV_BYTES = BN * D * 2;
+    static constexpr uint32_t P_BYTES = kBM * BN * 2;
+    static constexpr uint32_t BAR_OFF = Q_BYTES + 2 * kNS * KV_BYTES + P_BYTES;
+    static constexpr uint32_t NBAR = 1 + 2 * kNS + 2 + 1 + 1 + 1;
+    static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
+    static constexpr uint32_t TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+    static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, BN, false);
+    static constexpr uint32_t IDESC_PV = sm100::idesc_bf16(kBM, D, true);
+};
+
+template <int D, int BN>
+__global__ void __launch_bounds__(256, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, uint16_t *__restrict__ O,
+                      const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                      int H, int Hkv, int L, int Nb, float scale_log2) {
+    using C = TcCfg<D, BN>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sQ = smem_u32(base);
+    const uint32_t sK = sQ + C::Q_BYTES;
+    const uint32_t sV = sK + kNS * C::KV_BYTES;
+    const uint32_t sP = sV + kNS * C::KV_BYTES;
+    const uint32_t sBar = sQ + C::BAR_OFF;
+    const uint32_t q_full = sBar;
+    auto kv_full = [&](int s) { return sBar + 8u * (1 + s); };
+    auto kv_empty = [&](int s) { return sBar + 8u * (1 + kNS + s); };
+    auto s_full = [&](int b) { return sBar + 8u * (1 + 2 * kNS + b); };
+    const uint32_t p_full = sBar + 8u * (3 + 2 * kNS);
+    const uint32_t o_bar = sBar + 8u * (4 + 2 * kNS);
+    const uint32_t fin_bar = sBar + 8u * (5 + 2 * kNS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + C::BAR_OFF + C::NBAR * 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x;
+    const int I = Nb - 1 - (int)blockIdx.y;  // long rows first
+    const int g = h / (H / Hkv);
+    const long crow = (long)h * Nb + I;
+    const int e0 = row_ptr[crow];
+    const int n = row_ptr[crow + 1] - e0;
+
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(q_full, 1);
+        for (int s = 0; s < kNS; ++s) {
+            sm100::mbar_init(kv_full(s), 1);
+            sm100::mbar_init(kv_empty(s), 1);
+        }
+        sm100::mbar_init(s_full(0), 1);
+        sm100::mbar_init(s_full(1), 1);
+        sm100::mbar_init(p_full, 128);
+        sm100::mbar_init(o_bar, 1);
+        sm100::mbar_init(fin_bar, 1);
+        sm100::fence_mbar_init();
+    }
+    if (warp == 2) {
+        sm100::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- producer
+            sm100::prefetch_tmap(&tmQ);
+            sm100::prefetch_tmap(&tmK);
+            sm100::prefetch_tmap(&tmV);
+            sm100::mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+            for (int c = 0; c < C::DC; ++c)
+                sm100::tma_load_2d(sQ + c * kBM * 128, &tmQ, c * 64, h * L + I * BN, q_full);
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j < n; ++j) {
+                const int s = j % kNS;
+                if (!wait_bar(kv_empty(s), ((j / kNS) & 1) ^ 1)) {
+                    ok = false;
+                    break;
+                }
+                const int J = __ldg(col_idx + e0 + j);
+                sm100::mbar_arrive_expect_tx(kv_full(s), 2 * C::KV_BYTES);
+                for (int c = 0; c < C::DC; ++c) {
+                    sm100::tma_load_2d(sK + s * C::KV_BYTES + c * BN * 128, &tmK, c * 64, g * L + J * BN,
+                                       kv_full(s));
+                    sm100::tma_load_2d(sV + s * C::KV_BYTES + c * BN * 128, &tmV, c * 64, g * L + J * BN,
+                                       kv_full(s));
+                }
+                issued = j + 1;
+            }
+            if (!ok) {
+                atomicOr(&g_device_errors, kErrTimeoutProducer);
+                // let the copies already in flight land before the CTA's memory is released
+                wait_bar(q_full, 0);
+                for (int j = issued > kNS ? issued - kNS : 0; j < issued; ++j)
+                    wait_bar(kv_full(j % kNS), (j / kNS) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- MMA issuer
+            bool ok = wait_bar(q_full, 0);
+            sm100::tc_fence_after();
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % kNS, b = j & 1;
+                if (!wait_bar(kv_full(s), (j / kNS) & 1)) return false;
+                sm100::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int c = kk >> 2, w = kk & 3;
+                    const uint64_t ad = sm100::smem_desc_sw128(sQ + c * kBM * 128 + w * 32, 16, 1024);
+                    const uint64_t bd =
+                        sm100::smem_desc_sw128(sK + s * C::KV_BYTES + c * BN * 128 + w * 32, 16, 1024);
+                    sm100::mma_ss(tmem + b * BN, ad, bd, C::IDESC_S, kk > 0);
+                }
+                sm100::mma_commit(s_full(b));
+                return true;
+            };
+            if (ok && n > 0) ok = issue_s(0);
+            for (int j = 0; ok && j < n; ++j) {
+                if (j + 1 < n && !issue_s(j + 1)) {
+                    ok = false;
+                    break;
+                }
+                if (!wait_bar(p_full, j & 1)) {
+                    ok = false;
+                    break;
+                }
+                sm100::tc_fence_after();
+                const int s = j % kNS;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const int c = kk >> 2, w = kk & 3;
+                    const uint64_t ad = sm100::smem_desc_sw128(sP + c * kBM * 128 + w * 32, 16, 1024);
+                    const uint64_t bd =
+                        sm100::smem_desc_sw128(sV + s * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024);
+                    sm100::mma_ss(tmem + 2 * BN, ad, bd, C::IDESC_PV, (j > 0 || kk > 0));
+                }
+                sm100::mma_commit(o_bar);
+                sm100::mma_commit(kv_empty(s));
+            }
+            // every MMA issued must complete before the TMEM is released
+            sm100::mma_commit(fin_bar);
+            if (!wait_bar(fin_bar, 0)) ok = false;
+            if (!ok) atomicOr(&g_device_errors, kErrTimeoutMma);
+        }
+    } else if (warp >= 4) {
+        // -------------------------------------------------------------------- softmax
+        const int r = threadIdx.x - 128;  // query row within the tile = TMEM lane
+        const long qpos = (long)I * BN + r;
+        const uint32_t trow = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const int b = j & 1;
+            ok = __all_sync(0xffffffffu, wait_bar(s_full(b), (j >> 1) & 1));
+            if (!ok) break;
+            sm100::tc_fence_after();
+            const int J = __ldg(col_idx + e0 + j);
+            float sv[BN];
+#pragma unroll
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t rg[32];
+                sm100::tmem_ld32(trow + b * BN + cc * 32, rg);
+                sm100::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(rg[i]);
+            }
+            const long k0 = (long)J * BN;
+            const bool diag = (J == I);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < BN; ++i) {
+                float v = sv[i] * scale_log2;
+                if (diag && k0 + i > qpos) v = -INFINITY;
+                sv[i] = v;
+                mx = fmaxf(mx, v);
+            }
+            // P of the previous block is still being read (and O written) by the MMA
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, wait_bar(o_bar, (j - 1) & 1));
+                if (!ok) break;
+                sm100::tc_fence_after();
+            }
+            // Lazy rescale: a row keeps its stale max while p <= 2^8.  The decision is per row,
+            // but tcgen05.ld/st are warp-collective, so the O rescale runs for the whole warp
+            // whenever any of its rows needs it (alpha = 1 on the others).
+            const bool need = mx > m + 8.f;
+            const float alpha = need ? exp2f(m - mx) : 1.f;  // 0 on a row's first block
+            l *= alpha;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t rg[32];
+                    sm100::tmem_ld32(trow + 2 * BN + cc * 32, rg);
+                    sm100::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) rg[i] = __float_as_uint(__uint_as_float(rg[i]) * alpha);
+                    sm100::tmem_st32(trow + 2 * BN + cc * 32, rg);
+                }
+                sm100::tmem_wait_st();
+            }
+            if (need) m = mx;
+            const float mu = (m == -INFINITY) ? 0.f : m;  // a row with nothing attended yet
+            float rs = 0.f;
+            uint8_t *prow = base + (sP - sQ) + r * 128;
+#pragma unroll
+            for (int c16 = 0; c16 < BN / 8; ++c16) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = exp2f(sv[c16 * 8 + 2 * e] - mu);
+                    const float p1 = exp2f(sv[c16 * 8 + 2 * e + 1] - mu);
+                    rs += p0 + p1;
+                    pk[e] = pack_bf16(p0, p1);
+                }
+                const int kc = c16 >> 3, cw = c16 & 7;
+                *reinterpret_cast<uint4 *>(prow + kc * kBM * 128 + ((cw ^ (r & 7)) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            l += rs;
+            sm100::fence_proxy_async_smem();
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(p_full);
+        }
+        if (ok && n > 0) {
+            ok = __all_sync(0xffffffffu, wait_bar(o_bar, (n - 1) & 1));
+            sm100::tc_fence_after();
+        }
+        if (!ok) {
+            if (lane == 0) atomicOr(&g_device_errors, kErrTimeoutSoftmax);
+        } else {
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            uint16_t *orow = O + ((long)h * L + qpos) * D;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t rg[32];
+                sm100::tmem_ld32(trow + 2 * BN + cc * 32, rg);
+                sm100::tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16(__uint_as_float(rg[2 * i]) * inv, __uint_as_float(rg[2 * i + 1]) * inv);
+                if (r < BN) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
+            }
+        }
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 view [rows][d] of a row-major tensor, boxes of 64 columns x box_rows rows,
+// 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, int d, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BN>
+rr_status_t launch_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H, int Hkv, int L,
+                      const int32_t *row_ptr, const int32_t *col_idx, float scale, uint16_t *O,
+                      cudaStream_t st) {
+    using C = TcCfg<D, BN>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, Q, (uint64_t)H * L, D, kBM) || !make_map(&mk, K, (uint64_t)Hkv * L, D, BN) ||
+        !make_map(&mv, V, (uint64_t)Hkv * L, D, BN))
+        return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cuTensorMapEncodeTiled failed");
+    // at least 116 KB of shared memory: one CTA per SM, so TMEM allocation never contends
+    size_t smem = C::SMEM + 1024;
+    if (smem < 116 * 1024) smem = 116 * 1024;
+    auto kern = prefill_tc_kernel<D, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    const int Nb = L / BN;
+    dim3 grid(H, Nb);
+    kern<<<grid, 256, smem, st>>>(mq, mk, mv, O, row_ptr, col_idx, H, Hkv, L, Nb,
+                                  scale * 1.4426950408889634f);
+    return check_launch("rr_sparse_prefill: prefill_tc_kernel");
+}
+
+}  // namespace
+
+rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H, int Hkv,
+                              int L, int d, int B, const int32_t *row_ptr, const int32_t *col_idx,
+                              float scale, uint16_t *O, cudaStream_t st) {
+    if (d == 128 && B == 128) return launch_tc<128, 128>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
+    if (d == 128 && B == 64) return launch_tc<128, 64>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
+    if (d == 64 && B == 128) return launch_tc<64, 128>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
+    return launch_tc<64, 64>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
+}
+
+rr_status_t read_device_errors(unsigned *out, bool reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_errors, sizeof(unsigned));
+    if (e == cudaSuccess && reset) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_device_errors, &zero, sizeof(unsigned));
+    }
+    if (e != cudaSuccess)
+        return set_error(RR_ERR_CUDA, "rr_device_errors: %s", cudaGetErrorString(e));
+    return RR_OK;
+}
+
+}  // namespace rr

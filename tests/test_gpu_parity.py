@@ -49,6 +49,7 @@ def _gpu_pipeline(w, t, dev, tau=None, protect_last=True, strategy="head", layer
     rp, ci, nnz = rr.select(A, tau, protect_last)
     O = rr.sparse_prefill(Q, K, V, rp, ci, w.B)
     torch.cuda.synchronize()
+    assert rr.device_errors() == 0, "a kernel gave up a bounded wait"
     n = int(nnz.item())
     rp_h = rp.cpu().numpy()
     assert rp_h[-1] == n
@@ -178,6 +179,10 @@ def test_custom_scale_and_single_block(cuda_device):
     rows = [(h, q) for h in range(2) for q in range(64)]
     O_ref = oracle.prefill_rows(t["Q"], t["K"], t["V"], w.B, rp, ci, rows, scale=0.05)
     _check_output(O.float().cpu().reshape(-1, w.d).numpy(), O_ref)
+
+
+def test_no_device_errors_recorded(cuda_device):
+    assert rr.device_errors(reset=False) == 0
 
 
 def test_empty_sequence(cuda_device):
