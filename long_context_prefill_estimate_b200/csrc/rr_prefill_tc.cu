@@ -7,14 +7,17 @@
 // rows are padding that is computed and never stored).  The CTA walks only the CSR entries
 // of row h*Nb + I.  Warp roles:
 //   warp 0      TMA producer: Q tile once, then K and V tiles of each selected block into a
-//               2-stage ring (128-byte swizzle, mbarrier transaction counts).
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM buffers, then
-//               O += P_j V_j into a TMEM accumulator; completion signalled by tcgen05.commit.
+//               ring of 3-4 stages (128-byte swizzle, mbarrier transaction counts).
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T (both operands in shared memory) into
+//               one of two TMEM buffers, then O += P_j V_j with P_j read from TMEM (the
+//               A-from-tensor-memory form) and V_j from shared memory; completion is signalled
+//               by tcgen05.commit.
 //   warp 2      TMEM allocation / release.
-//   warps 4-7   softmax: one thread per query row (TMEM lane), online softmax in fp32 with a
-//               lazily rescaled running max (O is rescaled in TMEM only when the max grows by
-//               more than 2^8), P written to shared memory in the MMA operand layout, final
-//               normalisation and bf16 store.
+//   warps 4-7   softmax: one thread per query row (TMEM lane).  Online softmax in fp32 with a
+//               lazily rescaled running max (O is rescaled in TMEM only when a row's max grows
+//               by more than 2^8), P packed to bf16 pairs and stored back into TMEM, final
+//               normalisation and bf16 store of O.
+// TMEM columns: S0, S1 (fp32, B each), O (fp32, d), P (bf16 pairs, B/2).
 // K and V come from KV head h / (H/Hkv); the heads of a KV group run as adjacent CTAs so
 // their K/V tiles are served from L2.  Every wait is bounded (about one second of
 // %globaltimer); a timeout sets a device error bit and the CTA drains and exits.
@@ -50,21 +53,34 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
     }
 }
 
+// 2^x on the SFU (approximate, flushes denormals; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 constexpr int kBM = 128;  // query rows per CTA
-constexpr int kNS = 2;    // K/V pipeline stages
 
 template <int D, int BN>
 struct TcCfg {
-    static constexpr int DC = D / 64;                       // 64-element (128-byte) column chunks
+    static constexpr int DC = D / 64;  // 64-element (128-byte) column chunks
     static constexpr uint32_t Q_BYTES = kBM * D * 2;
     static constexpr uint32_t KV_BYTES = BN * D * 2;
-    static constexpr uint32_t P_BYTES = kBM * BN * 2;
-    static constexpr uint32_t BAR_OFF = Q_BYTES + 2 * kNS * KV_BYTES + P_BYTES;
-    static constexpr uint32_t NBAR = 1 + 2 * kNS + 2 + 1 + 1 + 1;
+    // as many K/V stages (up to 4) as fit next to Q in 225 KB of shared memory
+    static constexpr int NS_FIT = (int)((225u * 1024u - Q_BYTES - 1024u - 256u) / (2u * KV_BYTES));
+    static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+    static constexpr uint32_t BAR_OFF = Q_BYTES + 2 * NS * KV_BYTES;
+    static constexpr uint32_t NBAR = 1 + 2 * NS + 2 + 1 + 1 + 1;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
-    static constexpr uint32_t TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+    // TMEM columns: S0 [0,BN) S1 [BN,2BN) O [2BN,2BN+D) P [2BN+D, 2BN+D+BN/2) (bf16 pairs)
+    static constexpr uint32_t S_COL = 0, O_COL = 2 * BN, P_COL = 2 * BN + D;
+    static constexpr uint32_t TMEM_NEED = 2 * BN + D + BN / 2;
+    static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, BN, false);
     static constexpr uint32_t IDESC_PV = sm100::idesc_bf16(kBM, D, true);
+    static_assert(NS >= 2, "need at least two K/V stages");
+    static_assert(TMEM_NEED <= 512, "TMEM budget");
 };
 
 template <int D, int BN>
@@ -74,12 +90,12 @@ __global__ void __launch_bounds__(256, 1)
                       const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
                       int H, int Hkv, int L, int Nb, float scale_log2) {
     using C = TcCfg<D, BN>;
+    constexpr int kNS = C::NS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_u32(base);
     const uint32_t sK = sQ + C::Q_BYTES;
     const uint32_t sV = sK + kNS * C::KV_BYTES;
-    const uint32_t sP = sV + kNS * C::KV_BYTES;
     const uint32_t sBar = sQ + C::BAR_OFF;
     const uint32_t q_full = sBar;
     auto kv_full = [&](int s) { return sBar + 8u * (1 + s); };
@@ -170,7 +186,7 @@ __global__ void __launch_bounds__(256, 1)
                     const uint64_t ad = sm100::smem_desc_sw128(sQ + c * kBM * 128 + w * 32, 16, 1024);
                     const uint64_t bd =
                         sm100::smem_desc_sw128(sK + s * C::KV_BYTES + c * BN * 128 + w * 32, 16, 1024);
-                    sm100::mma_ss(tmem + b * BN, ad, bd, C::IDESC_S, kk > 0);
+                    sm100::mma_ss(tmem + C::S_COL + b * BN, ad, bd, C::IDESC_S, kk > 0);
                 }
                 sm100::mma_commit(s_full(b));
                 return true;
@@ -189,11 +205,10 @@ __global__ void __launch_bounds__(256, 1)
                 const int s = j % kNS;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const int c = kk >> 2, w = kk & 3;
-                    const uint64_t ad = sm100::smem_desc_sw128(sP + c * kBM * 128 + w * 32, 16, 1024);
                     const uint64_t bd =
                         sm100::smem_desc_sw128(sV + s * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024);
-                    sm100::mma_ss(tmem + 2 * BN, ad, bd, C::IDESC_PV, (j > 0 || kk > 0));
+                    sm100::mma_ts(tmem + C::O_COL, tmem + C::P_COL + kk * 8, bd, C::IDESC_PV,
+                                  (j > 0 || kk > 0));
                 }
                 sm100::mma_commit(o_bar);
                 sm100::mma_commit(kv_empty(s));
@@ -216,25 +231,25 @@ __global__ void __launch_bounds__(256, 1)
             if (!ok) break;
             sm100::tc_fence_after();
             const int J = __ldg(col_idx + e0 + j);
-            float sv[BN];
+            uint32_t sr[BN];
 #pragma unroll
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t rg[32];
-                sm100::tmem_ld32(trow + b * BN + cc * 32, rg);
-                sm100::tmem_wait_ld();
+            for (int cc = 0; cc < BN / 32; ++cc)
+                sm100::tmem_ld32(trow + C::S_COL + b * BN + cc * 32,
+                                 *reinterpret_cast<uint32_t(*)[32]>(sr + cc * 32));
+            sm100::tmem_wait_ld();
+            float mraw = -INFINITY;
+            if (J == I) {  // diagonal block: keys after the query row are masked
+                const int lim = r;  // key i of the block is visible iff i <= r
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(rg[i]);
+                for (int i = 0; i < BN; ++i) {
+                    if (i > lim) sr[i] = __float_as_uint(-INFINITY);
+                    mraw = fmaxf(mraw, __uint_as_float(sr[i]));
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < BN; ++i) mraw = fmaxf(mraw, __uint_as_float(sr[i]));
             }
-            const long k0 = (long)J * BN;
-            const bool diag = (J == I);
-            float mx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < BN; ++i) {
-                float v = sv[i] * scale_log2;
-                if (diag && k0 + i > qpos) v = -INFINITY;
-                sv[i] = v;
-                mx = fmaxf(mx, v);
-            }
+            const float mx = mraw * scale_log2;  // scale > 0 keeps the order
             // P of the previous block is still being read (and O written) by the MMA
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, wait_bar(o_bar, (j - 1) & 1));
@@ -251,34 +266,30 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t rg[32];
-                    sm100::tmem_ld32(trow + 2 * BN + cc * 32, rg);
+                    sm100::tmem_ld32(trow + C::O_COL + cc * 32, rg);
                     sm100::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) rg[i] = __float_as_uint(__uint_as_float(rg[i]) * alpha);
-                    sm100::tmem_st32(trow + 2 * BN + cc * 32, rg);
+                    sm100::tmem_st32(trow + C::O_COL + cc * 32, rg);
                 }
-                sm100::tmem_wait_st();
             }
             if (need) m = mx;
-            const float mu = (m == -INFINITY) ? 0.f : m;  // a row with nothing attended yet
+            const float nm = (m == -INFINITY) ? 0.f : -m;  // a row with nothing attended yet
             float rs = 0.f;
-            uint8_t *prow = base + (sP - sQ) + r * 128;
 #pragma unroll
-            for (int c16 = 0; c16 < BN / 8; ++c16) {
-                uint32_t pk[4];
+            for (int hc = 0; hc < BN / 64; ++hc) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(sv[c16 * 8 + 2 * e] - mu);
-                    const float p1 = exp2f(sv[c16 * 8 + 2 * e + 1] - mu);
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[hc * 64 + 2 * e]), scale_log2, nm));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[hc * 64 + 2 * e + 1]), scale_log2, nm));
                     rs += p0 + p1;
                     pk[e] = pack_bf16(p0, p1);
                 }
-                const int kc = c16 >> 3, cw = c16 & 7;
-                *reinterpret_cast<uint4 *>(prow + kc * kBM * 128 + ((cw ^ (r & 7)) << 4)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                sm100::tmem_st32(trow + C::P_COL + hc * 32, pk);
             }
+            sm100::tmem_wait_st();
             l += rs;
-            sm100::fence_proxy_async_smem();
             sm100::tc_fence_before();
             sm100::mbar_arrive(p_full);
         }
@@ -294,7 +305,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t rg[32];
-                sm100::tmem_ld32(trow + 2 * BN + cc * 32, rg);
+                sm100::tmem_ld32(trow + C::O_COL + cc * 32, rg);
                 sm100::tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
