@@ -15,9 +15,11 @@
 //   warp 2      TMEM allocation / release.
 //   warps 4-7   softmax: one thread per query row (TMEM lane).  Online softmax in fp32 with a
 //               lazily rescaled running max (O is rescaled in TMEM only when a row's max grows
-//               by more than 2^8), P packed to bf16 pairs and stored back into TMEM, final
+//               by more than 2^8), P packed to bf16 pairs and stored back into TMEM (two
+//               buffers, so block j's softmax never waits for block j-1's P*V), final
 //               normalisation and bf16 store of O.
-// TMEM columns: S0, S1 (fp32, B each), O (fp32, d), P (bf16 pairs, B/2).
+// TMEM columns: S0, S1 (fp32, B each), O (fp32, d), P0, P1 (bf16 pairs, B/2 each).
+// The producer also prefetches the K/V tiles of the next few selected blocks into L2.
 // K and V come from KV head h / (H/Hkv); the heads of a KV group run as adjacent CTAs so
 // their K/V tiles are served from L2.  Every wait is bounded (about one second of
 // %globaltimer); a timeout sets a device error bit and the CTA drains and exits.
@@ -60,6 +62,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Packed pairs of fp32 (one 64-bit register, two lanes of the FMA pipe per instruction).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 constexpr int kBM = 128;  // query rows per CTA
 
 template <int D, int BN>
@@ -68,14 +91,16 @@ struct TcCfg {
     static constexpr uint32_t Q_BYTES = kBM * D * 2;
     static constexpr uint32_t KV_BYTES = BN * D * 2;
     // as many K/V stages (up to 4) as fit next to Q in 225 KB of shared memory
+    static constexpr int PF = 4;  // K/V blocks prefetched into L2 ahead of the shared-memory loads
     static constexpr int NS_FIT = (int)((225u * 1024u - Q_BYTES - 1024u - 256u) / (2u * KV_BYTES));
     static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
     static constexpr uint32_t BAR_OFF = Q_BYTES + 2 * NS * KV_BYTES;
     static constexpr uint32_t NBAR = 1 + 2 * NS + 2 + 1 + 1 + 1;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
-    // TMEM columns: S0 [0,BN) S1 [BN,2BN) O [2BN,2BN+D) P [2BN+D, 2BN+D+BN/2) (bf16 pairs)
+    // TMEM columns: S0 [0,BN) S1 [BN,2BN) O [2BN,2BN+D) P0, P1 [2BN+D, 2BN+D+BN) (bf16 pairs,
+    // BN/2 columns each)
     static constexpr uint32_t S_COL = 0, O_COL = 2 * BN, P_COL = 2 * BN + D;
-    static constexpr uint32_t TMEM_NEED = 2 * BN + D + BN / 2;
+    static constexpr uint32_t TMEM_NEED = 2 * BN + D + BN;
     static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, BN, false);
     static constexpr uint32_t IDESC_PV = sm100::idesc_bf16(kBM, D, true);
@@ -107,9 +132,15 @@ __global__ void __launch_bounds__(256, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + C::BAR_OFF + C::NBAR * 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x;
-    const int I = Nb - 1 - (int)blockIdx.y;  // long rows first
-    const int g = h / (H / Hkv);
+    // Launch order: KV group by KV group, and inside a group query blocks from the longest
+    // CSR rows down with the group's heads adjacent.  CTAs resident at the same time then
+    // stream one KV head's K/V, which stays in L2.
+    const int G = H / Hkv;
+    const long lin = blockIdx.x;
+    const int g = (int)(lin / ((long)G * Nb));
+    const int within = (int)(lin % ((long)G * Nb));
+    const int I = Nb - 1 - within / G;
+    const int h = g * G + within % G;
     const long crow = (long)h * Nb + I;
     const int e0 = row_ptr[crow];
     const int n = row_ptr[crow + 1] - e0;
@@ -147,7 +178,21 @@ __global__ void __launch_bounds__(256, 1)
                 sm100::tma_load_2d(sQ + c * kBM * 128, &tmQ, c * 64, h * L + I * BN, q_full);
             int issued = 0;
             bool ok = true;
+            for (int j = 0; j < n && j < C::PF; ++j) {
+                const int Jp = __ldg(col_idx + e0 + j);
+                for (int c = 0; c < C::DC; ++c) {
+                    sm100::tma_prefetch_2d(&tmK, c * 64, g * L + Jp * BN);
+                    sm100::tma_prefetch_2d(&tmV, c * 64, g * L + Jp * BN);
+                }
+            }
             for (int j = 0; j < n; ++j) {
+                if (j + C::PF < n) {
+                    const int Jp = __ldg(col_idx + e0 + j + C::PF);
+                    for (int c = 0; c < C::DC; ++c) {
+                        sm100::tma_prefetch_2d(&tmK, c * 64, g * L + Jp * BN);
+                        sm100::tma_prefetch_2d(&tmV, c * 64, g * L + Jp * BN);
+                    }
+                }
                 const int s = j % kNS;
                 if (!wait_bar(kv_empty(s), ((j / kNS) & 1) ^ 1)) {
                     ok = false;
@@ -207,8 +252,8 @@ __global__ void __launch_bounds__(256, 1)
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bd =
                         sm100::smem_desc_sw128(sV + s * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024);
-                    sm100::mma_ts(tmem + C::O_COL, tmem + C::P_COL + kk * 8, bd, C::IDESC_PV,
-                                  (j > 0 || kk > 0));
+                    sm100::mma_ts(tmem + C::O_COL, tmem + C::P_COL + (j & 1) * (BN / 2) + kk * 8, bd,
+                                  C::IDESC_PV, (j > 0 || kk > 0));
                 }
                 sm100::mma_commit(o_bar);
                 sm100::mma_commit(kv_empty(s));
@@ -237,32 +282,34 @@ __global__ void __launch_bounds__(256, 1)
                 sm100::tmem_ld32(trow + C::S_COL + b * BN + cc * 32,
                                  *reinterpret_cast<uint32_t(*)[32]>(sr + cc * 32));
             sm100::tmem_wait_ld();
-            float mraw = -INFINITY;
-            if (J == I) {  // diagonal block: keys after the query row are masked
-                const int lim = r;  // key i of the block is visible iff i <= r
+            const bool diag = (J == I);
+            if (diag) {  // diagonal block: key i of the block is visible iff i <= r
 #pragma unroll
-                for (int i = 0; i < BN; ++i) {
-                    if (i > lim) sr[i] = __float_as_uint(-INFINITY);
-                    mraw = fmaxf(mraw, __uint_as_float(sr[i]));
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < BN; ++i) mraw = fmaxf(mraw, __uint_as_float(sr[i]));
+                for (int i = 0; i < BN; ++i)
+                    if (i > r) sr[i] = __float_as_uint(-INFINITY);
             }
+            float mq[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mq[k] = __uint_as_float(sr[k]);
+#pragma unroll
+            for (int i = 8; i < BN; ++i) mq[i & 7] = fmaxf(mq[i & 7], __uint_as_float(sr[i]));
+            const float mraw = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                                     fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
             const float mx = mraw * scale_log2;  // scale > 0 keeps the order
-            // P of the previous block is still being read (and O written) by the MMA
-            if (j > 0) {
+            // Lazy rescale: a row keeps its stale max while p <= 2^8.  The decision is per row,
+            // but tcgen05.ld/st are warp-collective, so the O rescale runs for the whole warp
+            // whenever any of its rows needs it (alpha = 1 on the others).  Only then must the
+            // previous block's P*V be complete; P itself is double-buffered.
+            const bool need = mx > m + 8.f;
+            float alpha = 1.f;
+            if (need) {
+                alpha = ex2_approx(m - mx);  // 0 on a row's first block
+                l *= alpha;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
                 ok = __all_sync(0xffffffffu, wait_bar(o_bar, (j - 1) & 1));
                 if (!ok) break;
                 sm100::tc_fence_after();
-            }
-            // Lazy rescale: a row keeps its stale max while p <= 2^8.  The decision is per row,
-            // but tcgen05.ld/st are warp-collective, so the O rescale runs for the whole warp
-            // whenever any of its rows needs it (alpha = 1 on the others).
-            const bool need = mx > m + 8.f;
-            const float alpha = need ? exp2f(m - mx) : 1.f;  // 0 on a row's first block
-            l *= alpha;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t rg[32];
@@ -275,19 +322,28 @@ __global__ void __launch_bounds__(256, 1)
             }
             if (need) m = mx;
             const float nm = (m == -INFINITY) ? 0.f : -m;  // a row with nothing attended yet
-            float rs = 0.f;
+            const f32x2 sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(nm, nm);
+            f32x2 rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int hc = 0; hc < BN / 64; ++hc) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[hc * 64 + 2 * e]), scale_log2, nm));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[hc * 64 + 2 * e + 1]), scale_log2, nm));
-                    rs += p0 + p1;
+                    const f32x2 x2 = f2_fma(f2_pack(__uint_as_float(sr[hc * 64 + 2 * e]),
+                                                    __uint_as_float(sr[hc * 64 + 2 * e + 1])),
+                                            sc2, nm2);
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    rs2[e & 1] = f2_add(rs2[e & 1], f2_pack(p0, p1));
                     pk[e] = pack_bf16(p0, p1);
                 }
-                sm100::tmem_st32(trow + C::P_COL + hc * 32, pk);
+                sm100::tmem_st32(trow + C::P_COL + (j & 1) * (BN / 2) + hc * 32, pk);
             }
+            float ra, rb, rc, rd;
+            f2_unpack(rs2[0], ra, rb);
+            f2_unpack(rs2[1], rc, rd);
+            const float rs = (ra + rb) + (rc + rd);
             sm100::tmem_wait_st();
             l += rs;
             sm100::tc_fence_before();
@@ -377,7 +433,7 @@ rr_status_t launch_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, i
     if (e != cudaSuccess)
         return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     const int Nb = L / BN;
-    dim3 grid(H, Nb);
+    dim3 grid((unsigned)((long)H * Nb));
     kern<<<grid, 256, smem, st>>>(mq, mk, mv, O, row_ptr, col_idx, H, Hkv, L, Nb,
                                   scale * 1.4426950408889634f);
     return check_launch("rr_sparse_prefill: prefill_tc_kernel");

@@ -181,6 +181,24 @@ def test_custom_scale_and_single_block(cuda_device):
     _check_output(O.float().cpu().reshape(-1, w.d).numpy(), O_ref)
 
 
+@pytest.mark.parametrize("scale", [1.5, 0.002])
+def test_extreme_softmax_scales(scale, cuda_device):
+    """A large scale spreads the logits far below the row max (exercising the clamped
+    exponential path); a tiny one makes the softmax nearly uniform."""
+    w = workloads.get(1, H=4, Hkv=1, L=2048)
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    A_gpu, rp, ci, _ = _gpu_pipeline(w, d, cuda_device)
+    O = rr.sparse_prefill(d["Q"], d["K"], d["V"], torch.from_numpy(rp).cuda(),
+                          torch.from_numpy(ci).cuda(), w.B, scale=scale)
+    torch.cuda.synchronize()
+    assert rr.device_errors() == 0
+    rows = [(h, q) for h in range(w.H) for q in range(0, w.L, 3)]
+    O_ref = oracle.prefill_rows(t["Q"], t["K"], t["V"], w.B, rp, ci, rows, scale=scale)
+    idx = torch.as_tensor(rows)
+    _check_output(O.float().cpu()[idx[:, 0], idx[:, 1]].numpy(), O_ref)
+
+
 def test_no_device_errors_recorded(cuda_device):
     assert rr.device_errors(reset=False) == 0
 
