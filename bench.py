@@ -106,14 +106,15 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_sample(w, t, n_rows: int, rng_seed: int = 0):
-    """Time the oracle on one query head's estimate + select and n_rows prefill rows of that
-    head; extrapolate linearly to the whole layer.  Returns (layer_seconds, info)."""
+def oracle_sample(w, t, n_rows: int, rng_seed: int = 0, n_est_heads: int = 1):
+    """Time the oracle on the estimate + select of query heads 0..n_est_heads-1 and on n_rows
+    prefill rows of head 0; extrapolate linearly to the whole layer.
+    Returns (layer_seconds, info)."""
     import oracle
 
     h = 0
     t0 = time.perf_counter()
-    A = oracle.estimate(t["Q"], t["K"], w.S, w.B, heads=(h, h + 1))
+    A = oracle.estimate(t["Q"], t["K"], w.S, w.B, heads=(0, n_est_heads))
     t1 = time.perf_counter()
     rp, ci = oracle.select(A[h:h + 1], w.tau, True)
     t2 = time.perf_counter()
@@ -123,7 +124,7 @@ def oracle_sample(w, t, n_rows: int, rng_seed: int = 0):
     rows = [(0, int(q)) for q in qs]
     oracle.prefill_rows(t["Q"][h:h + 1], t["K"][:1], t["V"][:1], w.B, rp, ci, rows)
     t3 = time.perf_counter()
-    est, sel, pre = t1 - t0, t2 - t1, t3 - t2
+    est, sel, pre = (t1 - t0) / n_est_heads, t2 - t1, t3 - t2
     # prefill cost grows with the number of attended keys: scale the sampled rows' time by
     # (keys attended by all rows of the head) / (keys attended by the sampled rows)
     B = w.B
@@ -307,15 +308,16 @@ def run_ours(args):
         line["dense_reference"] = dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_step)
     line["e2e"] = e2e(w, host, rr, torch, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
-        layer_s, info = oracle_sample(w, host, n_rows=args.cpu_rows)
+        layer_s, info = oracle_sample(w, host, n_rows=args.cpu_rows, n_est_heads=args.cpu_heads)
         import oracle
 
         line["cpu_baseline"] = {
             "value": dense / layer_s / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": (f"oracle estimate+select of query head 0 (all {w.Nb} query blocks) and "
-                       f"{args.cpu_rows} prefill rows of head 0, extrapolated linearly to the "
-                       f"layer ({layer_s:.1f} s/layer); measured {info['seconds_measured']:.1f} s"),
+            "sample": (f"oracle estimate of query heads 0..{args.cpu_heads - 1} (all {w.Nb} query "
+                       f"blocks each), select of head 0 and {args.cpu_rows} random prefill rows of "
+                       f"head 0, extrapolated linearly to the layer ({layer_s:.1f} s/layer); "
+                       f"measured {info['seconds_measured']:.1f} s"),
         }
     if world > 1:
         torch.distributed.barrier()
@@ -419,8 +421,9 @@ def main(argv=None):
     ap.add_argument("--L", type=int, default=0, help="override the sequence length")
     ap.add_argument("--quick", action="store_true", help="skip the tau sweep and dense comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=256)
-    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--cpu-rows", type=int, default=8192)
+    ap.add_argument("--cpu-heads", type=int, default=4)
+    ap.add_argument("--ref-rows", type=int, default=1024)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

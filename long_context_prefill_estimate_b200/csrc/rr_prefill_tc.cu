@@ -90,9 +90,10 @@ struct TcCfg {
     static constexpr int DC = D / 64;  // 64-element (128-byte) column chunks
     static constexpr uint32_t Q_BYTES = kBM * D * 2;
     static constexpr uint32_t KV_BYTES = BN * D * 2;
-    // as many K/V stages (up to 4) as fit next to Q in 225 KB of shared memory
+    // as many K/V stages (up to 4) as fit next to Q in the 227 KB a CTA may use (1024 bytes
+    // of alignment slack, 256 for barriers)
     static constexpr int PF = 4;  // K/V blocks prefetched into L2 ahead of the shared-memory loads
-    static constexpr int NS_FIT = (int)((225u * 1024u - Q_BYTES - 1024u - 256u) / (2u * KV_BYTES));
+    static constexpr int NS_FIT = (int)((227u * 1024u - Q_BYTES - 1024u - 256u) / (2u * KV_BYTES));
     static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
     static constexpr uint32_t BAR_OFF = Q_BYTES + 2 * NS * KV_BYTES;
     static constexpr uint32_t NBAR = 1 + 2 * NS + 2 + 1 + 1 + 1;
@@ -105,6 +106,7 @@ struct TcCfg {
     static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, BN, false);
     static constexpr uint32_t IDESC_PV = sm100::idesc_bf16(kBM, D, true);
     static_assert(NS >= 2, "need at least two K/V stages");
+    static_assert(SMEM + 1024 <= 227u * 1024u, "shared memory budget");
     static_assert(TMEM_NEED <= 512, "TMEM budget");
 };
 
