@@ -47,6 +47,29 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def prefill_traffic_per_launch(w):
+    """DRAM bytes per prefill launch from the committed ncu summary of the 32K Llama-shaped
+    layer, scaled by L (Q, K, V and O all grow linearly with L at fixed heads and d).  None
+    when the kernel source changed since the capture or the layer shape differs."""
+    import hashlib
+    import re
+
+    summ = os.path.join(ROOT, "profiles", "prefill_tc_llama3-8b-layer-L32k.md")
+    src = os.path.join(ROOT, "long_context_prefill_estimate_b200", "csrc", "rr_prefill_tc.cu")
+    if not (os.path.exists(summ) and os.path.exists(src)):
+        return None
+    text = open(summ).read()
+    m = re.search(r"prefill source sha256: ([0-9a-f]{16})", text)
+    rd = re.search(r"dram__bytes_read.sum / write.sum \| ([0-9.]+) MB / ([0-9.]+) MB", text)
+    if not (m and rd):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != m.group(1):
+        return None
+    if (w.H, w.Hkv, w.d, w.B) != (32, 8, 128, 128):
+        return None
+    return (float(rd.group(1)) + float(rd.group(2))) * 1e6 * w.L / 32768
+
+
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
         int(os.environ.get("LOCAL_RANK", "0"))
@@ -298,7 +321,9 @@ def run_ours(args):
                      "frac": prefill_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                      "frac_of_burst": prefill_tflops / peaks["bf16_tflops"],
                      "peak_source": f"{peak_kind} bf16 (sustained)",
-                     "flops_per_launch": sel_flops, "traffic": None},
+                     "flops_per_launch": sel_flops,
+                     "traffic": prefill_traffic_per_launch(w),
+                     "traffic_unit": "bytes/launch (ncu dram read+write at L=32768, scaled by L)"},
         "gpu_launches": 6 * args.steps,
         "clocks": clocks,
     }
