@@ -69,6 +69,13 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// 2^x on the SFU (relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 struct EstParams {
     const uint16_t *Q;
     const uint4 *frag;
@@ -172,19 +179,27 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
         const long col0 = (long)tile * 8 + 2 * tq;
 #pragma unroll
         for (int mm = 0; mm < MTW; ++mm) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            // four independent accumulation chains (hi/lo x two halves of the k-steps), summed
+            // afterwards, so consecutive MMAs do not wait on each other
+            float cq[4][4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cq[q][0] = cq[q][1] = cq[q][2] = cq[q][3] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-                mma_16816(c, a[mm][ks], b[ks].x, b[ks].y);
-                mma_16816(c, a[mm][ks], b[ks].z, b[ks].w);
+                const int hk = (2 * ks) / KS;
+                mma_16816(cq[2 * hk], a[mm][ks], b[ks].x, b[ks].y);
+                mma_16816(cq[2 * hk + 1], a[mm][ks], b[ks].z, b[ks].w);
             }
+            float c[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[e] = (cq[0][e] + cq[1][e]) + (cq[2][e] + cq[3][e]);
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 const float s0 = (col0 <= irow[mm][x]) ? c[2 * x] * p.c_log2 : -INFINITY;
                 const float s1 = (col0 + 1 <= irow[mm][x]) ? c[2 * x + 1] * p.c_log2 : -INFINITY;
                 const float mx = quad_max(fmaxf(s0, s1));
                 if (mx > mref[mm][x] + 8.f) {  // lazy rescale: stored sums stay <= r*2^8
-                    const float f = exp2f(mref[mm][x] - mx);  // 0 on the first block
+                    const float f = ex2_approx(mref[mm][x] - mx);  // 0 on the first block
                     lsum[mm][x] *= f;
                     bs[mm][x] *= f;
                     if (valid[mm][x]) {
@@ -193,7 +208,7 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
                     }
                     mref[mm][x] = mx;
                 }
-                bs[mm][x] += exp2f(s0 - mref[mm][x]) + exp2f(s1 - mref[mm][x]);
+                bs[mm][x] += ex2_approx(s0 - mref[mm][x]) + ex2_approx(s1 - mref[mm][x]);
             }
         }
         if (nt == p.NTB - 1) {
@@ -229,11 +244,11 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
         float l = 0.f;
         for (int w = 0; w < WJ; ++w) {
             const float m = stat_m[w * Rpad + x];
-            if (m != -INFINITY) l += stat_l[w * Rpad + x] * exp2f(m - M);
+            if (m != -INFINITY) l += stat_l[w * Rpad + x] * ex2_approx(m - M);
         }
         for (int w = 0; w < WJ; ++w) {
             const float m = stat_m[w * Rpad + x];
-            fac[w * Rpad + x] = (m != -INFINITY) ? exp2f(m - M) / l * inv_r : 0.f;
+            fac[w * Rpad + x] = (m != -INFINITY) ? ex2_approx(m - M) / l * inv_r : 0.f;
         }
     }
     __syncthreads();

@@ -3,8 +3,11 @@
 // (iii), Sec. 3.3 heading; the rule as the XAttention card states it: the smallest set of
 // blocks whose cumulative score reaches tau) with last-query-block protection (Sec. 4.3).
 //
-//   select_rows_kernel  one CTA per (head, query block) row: bitonic sort of the row's
-//                       causal scores on the key (score desc, J asc), float64 inclusive scan,
+//   select_rows_warp_kernel  one warp per row of up to 1024 causal blocks: the cut score by a
+//                       binary search over float bit patterns with float64 sums, ties at the
+//                       cut taken in ascending J; selected blocks as a bitmap.
+//   select_rows_kernel  one CTA per longer row: bitonic sort of the row's causal scores on the
+//                       key (score desc, J asc), float64 inclusive scan,
 //                       k* = 1 + #{k : cum_k < tau*T}, selected blocks as a bitmap.
 //   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr, nnz.
 //   emit_csr_kernel     one warp per row: bitmap -> ascending block indices in col_idx.
@@ -16,6 +19,8 @@ namespace rr {
 namespace {
 
 constexpr int kSelThreads = 256;
+// rows of up to 32*32 blocks go to the warp-per-row kernel, longer ones to the sorting kernel
+constexpr int kWarpRowSlots = 32;
 
 __device__ __forceinline__ uint64_t sort_key(float a, int J) {
     uint32_t bits = __float_as_uint(a);
@@ -55,8 +60,9 @@ __device__ double block_exclusive_scan(double v, double *warp_tot, double *total
 }
 
 __global__ void __launch_bounds__(kSelThreads)
-    select_rows_kernel(const float *__restrict__ A, int Nb, double tau, int protect_last, int P,
-                       int W, int *__restrict__ counts, uint32_t *__restrict__ bitmap) {
+    select_rows_kernel(const float *__restrict__ A, int Nb, long row_base, double tau,
+                       int protect_last, int P, int W, int *__restrict__ counts,
+                       uint32_t *__restrict__ bitmap) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);
     uint32_t *bm = reinterpret_cast<uint32_t *>(smem_raw + (size_t)P * 8);
@@ -64,8 +70,9 @@ __global__ void __launch_bounds__(kSelThreads)
     __shared__ double s_total;
     __shared__ int s_below;
 
-    const long row = blockIdx.x;
+    const long row = (long)blockIdx.x + row_base;
     const int I = (int)(row % Nb), n = I + 1, tid = threadIdx.x;
+    if (n <= 32 * kWarpRowSlots) return;  // handled by select_rows_warp_kernel
     uint32_t *out_bm = bitmap + row * W;
     const bool keep_all = (tau >= 1.0) || (protect_last && I == Nb - 1);
     if (keep_all) {
@@ -124,6 +131,122 @@ __global__ void __launch_bounds__(kSelThreads)
     __syncthreads();
     for (int w = tid; w < W; w += kSelThreads) out_bm[w] = bm[w];
     if (tid == 0) counts[row] = kstar;
+}
+
+// Warp per row for rows of at most 32*32 blocks (values held in registers, lane l owns blocks
+// J = l + 32*k).  The selected set is the first k* keys in (score desc, J asc) order; it is
+// found without sorting: s* = the largest score with sum_{a >= s*} a >= tau*T (binary search
+// over the bit patterns, which order non-negative floats), then all scores above s* plus the
+// ties at s* in ascending J until the sum reaches tau*T.  Sums in float64.
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__global__ void __launch_bounds__(256)
+    select_rows_warp_kernel(const float *__restrict__ A, int Nb, long nrows, double tau,
+                            int protect_last, int W, int *__restrict__ counts,
+                            uint32_t *__restrict__ bitmap) {
+    const long row = blockIdx.x * 8L + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= nrows) return;
+    const int I = (int)(row % Nb), n = I + 1;
+    if (n > 32 * kWarpRowSlots) return;  // long rows: select_rows_kernel
+    uint32_t *out_bm = bitmap + row * W;
+    const bool keep_all = (tau >= 1.0) || (protect_last && I == Nb - 1);
+    if (keep_all) {
+        for (int w = lane; w < W; w += 32) {
+            const int lo = w * 32;
+            uint32_t m = 0;
+            if (n >= lo + 32) m = 0xffffffffu;
+            else if (n > lo) m = (1u << (n - lo)) - 1u;
+            out_bm[w] = m;
+        }
+        if (lane == 0) counts[row] = n;
+        return;
+    }
+    const float *a = A + row * (long)Nb;
+    const int slots = (n + 31) >> 5;
+    uint32_t v[kWarpRowSlots];  // bit patterns (-0 as +0); 0 beyond the row
+    double tot = 0.0;
+    uint32_t vmax = 0;
+#pragma unroll
+    for (int k = 0; k < kWarpRowSlots; ++k) {
+        v[k] = 0;
+        if (k < slots) {
+            const int J = k * 32 + lane;
+            if (J < n) {
+                const float x = __ldg(a + J);
+                v[k] = (x == 0.f) ? 0u : __float_as_uint(x);
+                tot += (double)x;
+                vmax = max(vmax, v[k]);
+            }
+        }
+    }
+    const double T = warp_sum_d(tot);
+    const double thr = tau * T;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    // largest u in [0, vmax] with sum_{bits(a) >= u} a >= thr (true at u = 0)
+    uint32_t lo = 0, hi = vmax;
+    while (lo < hi) {
+        const uint32_t mid = lo + (hi - lo + 1) / 2;
+        double part = 0.0;
+#pragma unroll
+        for (int k = 0; k < kWarpRowSlots; ++k)
+            if (k < slots && v[k] >= mid) part += (double)__uint_as_float(v[k]);
+        if (warp_sum_d(part) >= thr) lo = mid;
+        else hi = mid - 1;
+    }
+    const uint32_t sbits = lo;
+    double gt = 0.0;
+    int cnt_gt = 0;
+#pragma unroll
+    for (int k = 0; k < kWarpRowSlots; ++k)
+        if (k < slots && v[k] > sbits) {
+            gt += (double)__uint_as_float(v[k]);
+            ++cnt_gt;
+        }
+    gt = warp_sum_d(gt);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt_gt += __shfl_xor_sync(0xffffffffu, cnt_gt, o);
+    // ties at s*, ascending J, until the running sum reaches thr (at least one block in all)
+    const double sval = (double)__uint_as_float(sbits);
+    int need_ties = 0;
+    {
+        double run = gt;
+        int take = 0;
+        // count of ties needed: smallest t >= 0 with gt + t*s >= thr (t >= 1 if no block yet)
+        if (!(run >= thr) || cnt_gt == 0) {
+            const double q = (sval > 0.0) ? ceil((thr - run) / sval) : 1.0;
+            take = (int)fmin(fmax(q, 1.0), 32.0 * kWarpRowSlots + 1.0);
+            if (take < 1) take = 1;
+            // guard the division against rounding: step until the sum rule holds exactly
+            while (take > 1 && run + (double)(take - 1) * sval >= thr) --take;
+            while (run + (double)take * sval < thr) ++take;
+        }
+        need_ties = take;
+    }
+    // emit the bitmap: blocks above s*, plus the first need_ties ties by ascending J
+    int taken = 0;
+    for (int w = lane; w < W; w += 32) out_bm[w] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < kWarpRowSlots; ++k) {
+        if (k >= slots) break;
+        const int J = k * 32 + lane;
+        const bool valid = J < n;
+        const bool above = valid && v[k] > sbits;
+        const bool tie = valid && v[k] == sbits;
+        const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+        const int before = __popc(tb & ((1u << lane) - 1u));
+        const bool take_tie = tie && (taken + before < need_ties);
+        taken += __popc(tb);
+        const uint32_t sel = __ballot_sync(0xffffffffu, above || take_tie);
+        if (lane == 0) out_bm[k] = sel;  // W >= slots; word k covers blocks 32k..32k+31
+    }
+    if (lane == 0) counts[row] = cnt_gt + min(need_ties, taken);
 }
 
 __global__ void __launch_bounds__(1024)
@@ -238,15 +361,21 @@ rr_status_t launch_select(const float *A, int H, int Nb, double tau, int protect
     const int P = pow2_at_least(Nb < 2 ? 2 : Nb);
     int *counts = static_cast<int *>(ws);
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + align_up(nrows * 4, 256));
-    const size_t smem = select_smem_bytes(Nb);
-    cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess)
-        return set_error(RR_ERR_CUDA, "rr_select: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    select_rows_kernel<<<(unsigned)nrows, kSelThreads, smem, st>>>(A, Nb, tau, protect_last, P, W,
-                                                                   counts, bitmap);
-    rr_status_t s = check_launch("rr_select: select_rows_kernel");
+    select_rows_warp_kernel<<<(unsigned)((nrows + 7) / 8), 256, 0, st>>>(A, Nb, nrows, tau, protect_last,
+                                                                        W, counts, bitmap);
+    rr_status_t s = check_launch("rr_select: select_rows_warp_kernel");
     if (s != RR_OK) return s;
+    if (Nb > 32 * kWarpRowSlots) {  // rows I >= 1024 of every head: sort-based kernel
+        const size_t smem = select_smem_bytes(Nb);
+        cudaError_t e = cudaFuncSetAttribute(select_rows_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return set_error(RR_ERR_CUDA, "rr_select: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        select_rows_kernel<<<(unsigned)nrows, kSelThreads, smem, st>>>(A, Nb, 0L, tau, protect_last, P,
+                                                                       W, counts, bitmap);
+        s = check_launch("rr_select: select_rows_kernel");
+        if (s != RR_OK) return s;
+    }
     scan_counts_kernel<<<1, 1024, 0, st>>>(counts, nrows, row_ptr, nnz_out);
     s = check_launch("rr_select: scan_counts_kernel");
     if (s != RR_OK) return s;
