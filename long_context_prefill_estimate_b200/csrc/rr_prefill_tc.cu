@@ -323,6 +323,9 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
             if (need) m = mx;
+            // P_j goes to the buffer P_{j-2} used.  Its P*V product is complete: S_j was issued
+            // after P_{j-2} V_{j-2}, and the commit behind S_j (which this warpgroup waited for
+            // before reading S_j) fires only once every earlier MMA of the issuing thread is done.
             const float nm = (m == -INFINITY) ? 0.f : -m;  // a row with nothing attended yet
             const f32x2 sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(nm, nm);
             f32x2 rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
