@@ -70,6 +70,24 @@ def prefill_traffic_per_launch(w):
     return (float(rd.group(1)) + float(rd.group(2))) * 1e6 * w.L / 32768
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank float across the process group (the value itself when the job
+    has one rank).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank processed flops_per_rank in the (max-over-ranks) ms."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
         int(os.environ.get("LOCAL_RANK", "0"))
@@ -278,11 +296,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clocks = clk.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     ms_step = total_ms / args.steps
     stage = {k: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
              for k, (a, b) in {"estimate_ms": (0, 1), "select_ms": (1, 2),
@@ -302,7 +316,7 @@ def run_ours(args):
     sel_bytes = 4 * w.H * w.Nb * w.Nb + 4 * (w.H * w.Nb + 1) + 4 * nnz
     line = {
         "metric": METRIC,
-        "value": world * dense / (ms_step * 1e-3) / 1e12,
+        "value": aggregate_tflops(world, dense, ms_step),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "ms_per_layer": ms_step,
@@ -424,14 +438,10 @@ def e2e(w, host, rr, torch, dev, args):
         rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, ws=ws, out=out)
     e1.record(st)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / n
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, dev)
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    return {"value": world * dense_causal_flops(w) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": aggregate_tflops(world, dense_causal_flops(w), ms), "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n}
 
