@@ -21,8 +21,8 @@
  *     nothing; a failed launch returns RR_ERR_CUDA.  rr_last_error() then holds a
  *     human-readable reason (per calling thread).  No kernel traps or asserts.
  *   - L = 0 is accepted by every call as an empty problem: nothing is launched.
- *   - Supported: d in {64, 128}; B in {64, 128}; 1 <= S <= B with B % S == 0 and
- *     (B/S) % 8 == 0; L % B == 0; H % Hkv == 0; L <= 2^20; H <= 256.
+ *   - Supported: d in {64, 128}; B in {64, 128}; 1 <= S <= B with B % S == 0 and B/S = 4
+ *     or a multiple of 8; (L/S) % 8 == 0; L % B == 0; H % Hkv == 0; L <= 2^20; H <= 256.
  */
 #ifndef RR_ATTN_H
 #define RR_ATTN_H

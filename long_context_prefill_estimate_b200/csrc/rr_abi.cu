@@ -122,8 +122,10 @@ rr_status_t rr_estimate_strategy(const rr_bf16_t *Q, const rr_bf16_t *K, int H, 
     RR_TRY(check_common(fn, H, Hkv, L, d, B));
     if (S <= 0 || S > B || B % S)
         return set_error(RR_ERR_INVALID_ARG, "%s: stride S=%d must divide B=%d", fn, S, B);
-    if ((B / S) % 8)
-        return set_error(RR_ERR_UNSUPPORTED, "%s: B/S=%d must be a multiple of 8", fn, B / S);
+    if ((B / S) % 8 && B / S != 4)
+        return set_error(RR_ERR_UNSUPPORTED, "%s: B/S=%d must be 4 or a multiple of 8", fn, B / S);
+    if ((L / S) % 8)
+        return set_error(RR_ERR_UNSUPPORTED, "%s: L/S=%d strides must be a multiple of 8", fn, L / S);
     if ((int)strategy < RR_HEAD || (int)strategy > RR_HYBRID || layer < 0)
         return set_error(RR_ERR_INVALID_ARG, "%s: bad strategy %d / layer %d", fn, (int)strategy, layer);
     if (L == 0) return RR_OK;

@@ -80,7 +80,7 @@ struct EstParams {
     const uint16_t *Q;
     const uint4 *frag;
     float *A;
-    int H, L, S, r, Nb, NT, NTB;
+    int H, L, S, r, Nb, NT, NTB, BPT;  // NTB: 8-stride tiles per work group, BPT: blocks per group
     int G, hc, nHC, R, MT, MTW, NG, WJ;
     int mode, layer;
     float c_log2;  // log2(e) / (S * sqrt(d))
@@ -95,7 +95,7 @@ __device__ __forceinline__ int rr_offset(int h, int S, int mode, int layer) {
     }
 }
 
-template <int D, int MTW>
+template <int D, int MTW, int BPT>
 __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParams p) {
     constexpr int KS = D / 16;
     constexpr int QSTRIDE = D + 8;  // bf16 elements per staged query row (16-byte pad)
@@ -156,7 +156,10 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
             bs[mm][x] = 0.f;
         }
 
-    const int nJ = (I >= jw) ? (I - jw) / WJ + 1 : 0;  // J = jw, jw+WJ, ... <= I
+    // Work groups: for r >= 8 a group is one key block (r/8 stride tiles); for r = 4 it is one
+    // stride tile spanning two key blocks.  Warp jw takes groups jw, jw+WJ, ...
+    const int ngroups = (I + BPT) / BPT;  // groups covering blocks 0..I
+    const int nJ = (ngroups > jw) ? (ngroups - 1 - jw) / WJ + 1 : 0;
     const int nunits = nJ * p.NTB;
     const uint4 *fragg = p.frag + (long)g * p.NT * KS * 32 + lane;
     uint4 b[KS], bn[KS];
@@ -166,13 +169,13 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
         for (int ks = 0; ks < KS; ++ks) bn[ks] = __ldg(src + ks * 32);
     }
     for (int u = 0; u < nunits; ++u) {
-        const int J = jw + (u / p.NTB) * WJ, nt = u % p.NTB;
-        const int tile = J * p.NTB + nt;
+        const int grpi = jw + (u / p.NTB) * WJ, nt = u % p.NTB;
+        const int tile = grpi * p.NTB + nt;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) b[ks] = bn[ks];
         if (u + 1 < nunits) {
-            const int J2 = jw + ((u + 1) / p.NTB) * WJ, nt2 = (u + 1) % p.NTB;
-            const uint4 *src = fragg + (long)(J2 * p.NTB + nt2) * KS * 32;
+            const int g2 = jw + ((u + 1) / p.NTB) * WJ, nt2 = (u + 1) % p.NTB;
+            const uint4 *src = fragg + (long)(g2 * p.NTB + nt2) * KS * 32;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) bn[ks] = __ldg(src + ks * 32);
         }
@@ -204,7 +207,11 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
                     bs[mm][x] *= f;
                     if (valid[mm][x]) {
                         float *row = sst + (long)rho[mm][x] * Nb;
-                        for (int k = tq; k < u / p.NTB; k += 4) row[jw + k * WJ] *= f;
+                        const int done = u / p.NTB;  // this warp's groups already stored
+                        for (int k = tq; k < done * BPT; k += 4) {
+                            const int J = (jw + (k / BPT) * WJ) * BPT + k % BPT;
+                            if (J < Nb) row[J] *= f;
+                        }
                     }
                     mref[mm][x] = mx;
                 }
@@ -217,10 +224,23 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
             for (int mm = 0; mm < MTW; ++mm)
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    const float tot = quad_sum(bs[mm][x]);
+                    float tot;
+                    int J;
+                    bool writer;
+                    if constexpr (BPT == 1) {  // the quad's 8 columns are one block
+                        tot = quad_sum(bs[mm][x]);
+                        J = grpi;
+                        writer = (tq == 0);
+                    } else {  // columns 0-3 (lanes 0,1) and 4-7 (lanes 2,3) are two blocks
+                        tot = bs[mm][x] + __shfl_xor_sync(0xffffffffu, bs[mm][x], 1);
+                        J = grpi * 2 + (tq >> 1);
+                        writer = ((tq & 1) == 0);
+                    }
                     bs[mm][x] = 0.f;
-                    lsum[mm][x] += tot;
-                    if (tq == 0 && valid[mm][x]) sst[(long)rho[mm][x] * Nb + J] = tot;
+                    // the row sum takes each block once: add the other half's share too
+                    if constexpr (BPT == 1) lsum[mm][x] += tot;
+                    else lsum[mm][x] += tot + __shfl_xor_sync(0xffffffffu, tot, 2);
+                    if (writer && valid[mm][x] && J <= I) sst[(long)rho[mm][x] * Nb + J] = tot;
                 }
             __syncwarp();
         }
@@ -259,7 +279,7 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
         for (int J = tid; J < Nb; J += kEstThreads) {
             float v = 0.f;
             if (J <= I) {
-                const int w = J % WJ;
+                const int w = (J / BPT) % WJ;
                 for (int ii = 0; ii < r; ++ii) {
                     const int x = hh * r + ii;
                     v += sst[(long)x * Nb + J] * fac[w * Rpad + x];
@@ -342,7 +362,8 @@ rr_status_t launch_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv
     p.r = B / S;
     p.Nb = Nb;
     p.NT = Ns / 8;
-    p.NTB = p.r / 8;
+    p.NTB = p.r >= 8 ? p.r / 8 : 1;
+    p.BPT = p.r >= 8 ? 1 : 8 / p.r;
     p.G = H / Hkv;
     p.hc = pl.hc;
     p.nHC = pl.nHC;
@@ -364,9 +385,14 @@ rr_status_t launch_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv
         kern<<<grid, kEstThreads, pl.smem, st>>>(p);
         return check_launch("rr_estimate: estimate_kernel");
     };
+    if (p.BPT == 1) {
+        if (d == 128)
+            return pl.MTW == 2 ? launch(estimate_kernel<128, 2, 1>) : launch(estimate_kernel<128, 1, 1>);
+        return pl.MTW == 2 ? launch(estimate_kernel<64, 2, 1>) : launch(estimate_kernel<64, 1, 1>);
+    }
     if (d == 128)
-        return pl.MTW == 2 ? launch(estimate_kernel<128, 2>) : launch(estimate_kernel<128, 1>);
-    return pl.MTW == 2 ? launch(estimate_kernel<64, 2>) : launch(estimate_kernel<64, 1>);
+        return pl.MTW == 2 ? launch(estimate_kernel<128, 2, 2>) : launch(estimate_kernel<128, 1, 2>);
+    return pl.MTW == 2 ? launch(estimate_kernel<64, 2, 2>) : launch(estimate_kernel<64, 1, 2>);
 }
 
 }  // namespace rr

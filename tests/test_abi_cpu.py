@@ -66,7 +66,8 @@ def test_estimate_rejections(L):
     assert _est(L, B=32) == UNSUPPORTED
     assert _est(L, Len=200) == UNSUPPORTED
     assert _est(L, S=3) == INVALID
-    assert _est(L, S=16) == UNSUPPORTED        # B/S = 4 is not a multiple of 8
+    assert _est(L, S=32) == UNSUPPORTED        # B/S = 2 is neither 4 nor a multiple of 8
+    assert _est(L, Len=64, S=16) == UNSUPPORTED  # L/S = 4 strides, not a multiple of 8
     assert _est(L, strategy=7) == INVALID
     assert _est(L, q=0) == INVALID
     assert _est(L, k=FAKE + 4) == INVALID      # misaligned

@@ -84,6 +84,8 @@ SMALL = [
     ("mha-s8-b128", workloads.get(0, H=4, Hkv=4, L=2048, d=128, S=8, B=128)),
     ("s1-b64", workloads.get(0, H=2, Hkv=1, L=512, d=64, S=1, B=64)),
     ("gqa7-d64", workloads.get(4, H=14, Hkv=2, L=4096, d=64, S=8, B=64, frame_len=512)),
+    ("s32-b128", workloads.get(1, H=8, Hkv=2, L=4096, S=32)),      # B/S = 4: two blocks per tile
+    ("s16-b64", workloads.get(0, L=2176, S=16, B=64)),              # B/S = 4 at B = 64
 ]
 
 
@@ -269,3 +271,34 @@ def test_full_size_sampled(idx, w, cuda_device):
     O_ref = oracle.prefill_rows(t["Q"], t["K"], t["V"], w.B, rp, ci, rows)
     idx_t = torch.as_tensor(rows, device=O.device)
     _check_output(O[idx_t[:, 0], idx_t[:, 1]].float().cpu().numpy(), O_ref)
+
+
+def test_selection_accuracy_diagnostic(cuda_device):
+    """RR selection vs the exact-mass (S = 1) selection: the GPU diagnostic equals the same
+    metrics computed from oracle scores and oracle selections."""
+    from long_context_prefill_estimate_b200 import diagnostics
+
+    w = workloads.get(1, H=4, Hkv=2, L=2048)
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    res = diagnostics.selection_accuracy(d["Q"], d["K"], w.S, w.B, w.tau)
+    A_rr = oracle.estimate(t["Q"], t["K"], w.S, w.B)
+    A_ex = oracle.estimate(t["Q"], t["K"], 1, w.B)
+    rp1, ci1, dg1 = oracle.select(A_rr, w.tau, True, diag=True)
+    rp2, ci2, dg2 = oracle.select(A_ex, w.tau, True, diag=True)
+    if _boundary_rows(dg1).any() or _boundary_rows(dg2).any():
+        pytest.skip("a selection boundary row makes the masks legitimately differ")
+    H, Nb = w.H, w.Nb
+    sel = np.zeros((H, Nb, Nb), bool)
+    ref = np.zeros((H, Nb, Nb), bool)
+    for r in range(H * Nb):
+        sel[r // Nb, r % Nb, ci1[rp1[r]:rp1[r + 1]]] = True
+        ref[r // Nb, r % Nb, ci2[rp2[r]:rp2[r + 1]]] = True
+    for h in range(H):
+        inter = (sel[h] & ref[h]).sum()
+        prec, rec = inter / sel[h].sum(), inter / ref[h].sum()
+        assert res["per_head"]["precision"][h] == pytest.approx(prec, abs=1e-12)
+        assert res["per_head"]["recall"][h] == pytest.approx(rec, abs=1e-12)
+        assert res["per_head"]["f1"][h] == pytest.approx(2 * prec * rec / (prec + rec), abs=1e-12)
+        cap = (A_ex[h] * sel[h]).sum(-1).mean()
+        assert res["per_head"]["captured_mass"][h] == pytest.approx(cap, abs=1e-5)
