@@ -423,7 +423,8 @@ def dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_sparse):
 
 def e2e(w, host, rr, torch, dev, args):
     """Same layer through the public API from pinned host buffers: H2D of Q/K/V, the three
-    stages, D2H of O, every step inside the timed region."""
+    stages, D2H of O, every step inside the timed region (the API overlaps the copies of one
+    slice of KV groups with the compute of another)."""
     pinned = {k: v.pin_memory() for k, v in host.items()}
     out = torch.empty(pinned["Q"].shape, dtype=torch.bfloat16, pin_memory=True)
     ws = rr.Workspace(w.H, w.Hkv, w.L, w.d, w.S, w.B, device=dev)
@@ -443,7 +444,9 @@ def e2e(w, host, rr, torch, dev, args):
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     return {"value": aggregate_tflops(world, dense_causal_flops(w), ms), "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n}
+            "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n,
+            "pipeline": f"{rr.default_chunks(w.Hkv)} slices of whole KV groups; copy-in, compute "
+                        f"and copy-out on three streams"}
 
 
 def main(argv=None):

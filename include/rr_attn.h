@@ -81,6 +81,24 @@ rr_status_t rr_estimate_strategy(const rr_bf16_t *Q, const rr_bf16_t *K, int H, 
                                  float *block_scores, void *workspace, size_t workspace_bytes,
                                  rr_stream_t stream);
 
+/*
+ * rr_estimate_heads -- rr_estimate_strategy for a slice of whole KV groups of a layer.
+ *
+ * Every step of the estimate is independent per query head, so a layer may be processed in
+ * slices (a pipeline over host copies, or KV groups sharded across GPUs).  Q points at the
+ * slice's first query head and K at its first KV head; H and Hkv are the slice's counts (the
+ * slice must hold whole KV groups, so the GQA mapping inside it is the layer's).  head_base is
+ * the layer-wide index of the slice's first query head: the round-robin offset of local head h
+ * is that of head head_base + h (HEAD: (head_base + h) mod S; HYBRID: (head_base + h + layer)
+ * mod S), so the slice's block_scores equal rows [head_base, head_base + H) of the whole
+ * layer's.  0 <= head_base <= 2^20, else RR_ERR_INVALID_ARG.  The page defines no slicing;
+ * this entry point only carries the head index across the cut.
+ */
+rr_status_t rr_estimate_heads(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L, int d,
+                              int S, int B, rr_strategy_t strategy, int layer, int head_base,
+                              float *block_scores, void *workspace, size_t workspace_bytes,
+                              rr_stream_t stream);
+
 /* Bytes of device workspace rr_select needs for H heads and Nb blocks per row. */
 size_t rr_select_workspace_bytes(int H, int Nb);
 

@@ -22,14 +22,15 @@ import torch
 
 __all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
            "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
-           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors"]
+           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors", "default_chunks"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "librrattn.so")
 
 STRATEGIES = {"head": 0, "none": 1, "layer": 2, "hybrid": 3}
 
-EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_workspace_bytes",
+EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_heads",
+                    "rr_estimate_workspace_bytes",
                     "rr_select", "rr_select_workspace_bytes", "rr_select_noalloc",
                     "rr_sparse_prefill",
                     "rr_validate_csr", "rr_device_errors", "rr_status_string", "rr_last_error",
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
     L.rr_estimate.restype = I
     L.rr_estimate_strategy.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P, Z, P]
     L.rr_estimate_strategy.restype = I
+    L.rr_estimate_heads.argtypes = [P, P, I, I, I, I, I, I, I, I, I, P, P, Z, P]
+    L.rr_estimate_heads.restype = I
     L.rr_select_workspace_bytes.argtypes = [I, I]
     L.rr_select_workspace_bytes.restype = Z
     L.rr_select.argtypes = [P, I, I, D, I, P, P, I64, P, P, Z, P]
@@ -134,8 +137,11 @@ class Workspace:
 
 def estimate(Q: torch.Tensor, K: torch.Tensor, S: int, B: int, strategy: str = "head",
              layer: int = 0, out: Optional[torch.Tensor] = None,
-             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Block importance [H][L/B][L/B] (float32) from round-robin sampled queries."""
+             workspace: Optional[torch.Tensor] = None, head_base: int = 0) -> torch.Tensor:
+    """Block importance [H][L/B][L/B] (float32) from round-robin sampled queries.
+
+    Q and K may be a slice of whole KV groups of a larger layer; head_base is then the
+    layer-wide index of Q's first head (it sets the round-robin offsets)."""
     _need_cuda("rr_estimate", Q, torch.bfloat16)
     _need_cuda("rr_estimate", K, torch.bfloat16)
     H, L, d = Q.shape
@@ -148,8 +154,8 @@ def estimate(Q: torch.Tensor, K: torch.Tensor, S: int, B: int, strategy: str = "
     need = estimate_workspace_bytes(H, Hkv, L, d, S, B)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=Q.device)
-    _check("rr_estimate", lib().rr_estimate_strategy(
-        _ptr(Q), _ptr(K), H, Hkv, L, d, S, B, STRATEGIES[strategy], layer, _ptr(out),
+    _check("rr_estimate", lib().rr_estimate_heads(
+        _ptr(Q), _ptr(K), H, Hkv, L, d, S, B, STRATEGIES[strategy], layer, head_base, _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(Q.device)))
     return out
 
@@ -204,12 +210,22 @@ def sparse_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: t
 def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, tau: float,
             protect_last: bool = True, strategy: str = "head", layer: int = 0,
             scale: Optional[float] = None, ws: Optional[Workspace] = None,
-            out: Optional[torch.Tensor] = None, return_intermediates: bool = False):
+            out: Optional[torch.Tensor] = None, return_intermediates: bool = False,
+            chunks: Optional[int] = None):
     """One attention layer's sparse prefill: estimate -> select -> sparse attention.
 
-    Host (CPU) tensors are accepted: they are copied to the current CUDA device and the
-    output is copied back (pinned host memory makes those copies asynchronous)."""
+    Host (CPU) tensors are accepted: the layer is then processed in `chunks` slices of whole
+    KV groups (default: the largest divisor of Hkv that is at most 8), each slice's inputs
+    copied in on one stream while the previous slice computes and the one before is copied
+    back on a third, and the call returns once O is on the host.  Pinned host memory makes
+    the copies asynchronous.  The result is identical to the one-pass device call: every
+    stage is independent per query head, and each slice is estimated with its layer-wide
+    head index.  The host path allocates its own slice-sized workspace (`ws` applies to the
+    device path); with return_intermediates it runs as one slice."""
     host = not Q.is_cuda
+    if host and not return_intermediates:
+        return _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, scale,
+                                       out, chunks)
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
         Q, K, V = (t.to(dev, non_blocking=True) for t in (Q, K, V))
@@ -230,6 +246,66 @@ def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, t
     if return_intermediates:
         return O, ws
     return O
+
+
+def default_chunks(Hkv: int) -> int:
+    """Slices of the host pipeline: the largest divisor of Hkv that is at most 8."""
+    return max(c for c in range(1, min(Hkv, 8) + 1) if Hkv % c == 0)
+
+
+def _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, scale, out, chunks):
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise RRAttnError("prefill", 1, f"{n}: host path needs contiguous bf16 CPU tensors")
+    H, L, d = Q.shape
+    Hkv = K.shape[0]
+    if Hkv <= 0 or H % Hkv or K.shape != (Hkv, L, d) or V.shape != K.shape:
+        raise RRAttnError("prefill", 1, f"shapes Q {tuple(Q.shape)} K {tuple(K.shape)} V {tuple(V.shape)}")
+    n = default_chunks(Hkv) if chunks is None else int(chunks)
+    if n <= 0 or Hkv % n:
+        raise RRAttnError("prefill", 1, f"chunks={n} must divide Hkv={Hkv}")
+    dst = out if out is not None else torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+    if dst.shape != Q.shape or dst.dtype != Q.dtype or dst.is_cuda or not dst.is_contiguous():
+        raise RRAttnError("prefill", 1, "out must be a contiguous bf16 host tensor shaped like Q")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gc, hc = Hkv // n, H // n
+    compute = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    Qd, Kd, Vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (Q, K, V))
+    Od = torch.empty(Q.shape, dtype=Q.dtype, device=dev)
+    ws = Workspace(hc, gc, L, d, S, B, device=dev)
+    # the fresh buffers may reuse memory last used on the compute stream
+    s_in.wait_stream(compute)
+    s_out.wait_stream(compute)
+    loaded = []
+    with torch.cuda.stream(s_in):
+        for c in range(n):
+            hs, gs = slice(c * hc, (c + 1) * hc), slice(c * gc, (c + 1) * gc)
+            Qd[hs].copy_(Q[hs], non_blocking=True)
+            Kd[gs].copy_(K[gs], non_blocking=True)
+            Vd[gs].copy_(V[gs], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            loaded.append(ev)
+    for c in range(n):
+        hs, gs = slice(c * hc, (c + 1) * hc), slice(c * gc, (c + 1) * gc)
+        compute.wait_event(loaded[c])
+        estimate(Qd[hs], Kd[gs], S, B, strategy=strategy, layer=layer, out=ws.block_scores,
+                 workspace=ws.est, head_base=c * hc)
+        select(ws.block_scores, tau, protect_last, row_ptr=ws.row_ptr, col_idx=ws.col_idx,
+               nnz=ws.nnz, workspace=ws.sel)
+        sparse_prefill(Qd[hs], Kd[gs], Vd[gs], ws.row_ptr, ws.col_idx, B, scale=scale, out=Od[hs])
+        done = torch.cuda.Event()
+        done.record(compute)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            dst[hs].copy_(Od[hs], non_blocking=True)
+    s_out.synchronize()
+    # every copy and kernel above has completed; later work on the compute stream may
+    # reuse the buffers
+    compute.wait_stream(s_in)
+    compute.wait_stream(s_out)
+    return dst
 
 
 def validate_csr(row_ptr: torch.Tensor, col_idx: torch.Tensor, H: int, Nb: int) -> int:

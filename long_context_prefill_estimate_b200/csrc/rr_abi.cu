@@ -12,7 +12,7 @@ namespace rr {
 size_t estimate_workspace_bytes(int Hkv, int L, int d, int S);
 bool estimate_supported(int H, int Hkv, int d, int S, int B, int L);
 rr_status_t launch_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, int d,
-                            int S, int B, int mode, int layer, float *A, void *ws,
+                            int S, int B, int mode, int layer, int head_base, float *A, void *ws,
                             cudaStream_t st);
 size_t select_workspace_bytes(int H, int Nb);
 rr_status_t launch_select(const float *A, int H, int Nb, double tau, int protect_last,
@@ -113,10 +113,10 @@ size_t rr_estimate_workspace_bytes(int H, int Hkv, int L, int d, int S, int B) {
     return estimate_workspace_bytes(Hkv, L, d, S);
 }
 
-rr_status_t rr_estimate_strategy(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L,
-                                 int d, int S, int B, rr_strategy_t strategy, int layer,
-                                 float *block_scores, void *workspace, size_t workspace_bytes,
-                                 rr_stream_t stream) {
+rr_status_t rr_estimate_heads(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L, int d,
+                              int S, int B, rr_strategy_t strategy, int layer, int head_base,
+                              float *block_scores, void *workspace, size_t workspace_bytes,
+                              rr_stream_t stream) {
     static const char *fn = "rr_estimate";
     g_last_error[0] = 0;
     RR_TRY(check_common(fn, H, Hkv, L, d, B));
@@ -126,8 +126,10 @@ rr_status_t rr_estimate_strategy(const rr_bf16_t *Q, const rr_bf16_t *K, int H, 
         return set_error(RR_ERR_UNSUPPORTED, "%s: B/S=%d must be 4 or a multiple of 8", fn, B / S);
     if ((L / S) % 8)
         return set_error(RR_ERR_UNSUPPORTED, "%s: L/S=%d strides must be a multiple of 8", fn, L / S);
-    if ((int)strategy < RR_HEAD || (int)strategy > RR_HYBRID || layer < 0)
-        return set_error(RR_ERR_INVALID_ARG, "%s: bad strategy %d / layer %d", fn, (int)strategy, layer);
+    if ((int)strategy < RR_HEAD || (int)strategy > RR_HYBRID || layer < 0 || head_base < 0 ||
+        head_base > (1 << 20))
+        return set_error(RR_ERR_INVALID_ARG, "%s: bad strategy %d / layer %d / head_base %d", fn,
+                         (int)strategy, layer, head_base);
     if (L == 0) return RR_OK;
     RR_TRY(check_ptr(fn, "Q", Q));
     RR_TRY(check_ptr(fn, "K", K));
@@ -140,8 +142,16 @@ rr_status_t rr_estimate_strategy(const rr_bf16_t *Q, const rr_bf16_t *K, int H, 
     if (!estimate_supported(H, Hkv, d, S, B, L))
         return set_error(RR_ERR_UNSUPPORTED, "%s: no launch plan fits (H=%d Hkv=%d L=%d S=%d B=%d)",
                          fn, H, Hkv, L, S, B);
-    return launch_estimate(Q, K, H, Hkv, L, d, S, B, (int)strategy, layer, block_scores, workspace,
-                           static_cast<cudaStream_t>(stream));
+    return launch_estimate(Q, K, H, Hkv, L, d, S, B, (int)strategy, layer, head_base, block_scores,
+                           workspace, static_cast<cudaStream_t>(stream));
+}
+
+rr_status_t rr_estimate_strategy(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L,
+                                 int d, int S, int B, rr_strategy_t strategy, int layer,
+                                 float *block_scores, void *workspace, size_t workspace_bytes,
+                                 rr_stream_t stream) {
+    return rr_estimate_heads(Q, K, H, Hkv, L, d, S, B, strategy, layer, 0, block_scores, workspace,
+                             workspace_bytes, stream);
 }
 
 rr_status_t rr_estimate(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L, int d,

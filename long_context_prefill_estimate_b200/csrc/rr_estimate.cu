@@ -83,6 +83,7 @@ struct EstParams {
     int H, L, S, r, Nb, NT, NTB, BPT;  // NTB: 8-stride tiles per work group, BPT: blocks per group
     int G, hc, nHC, R, MT, MTW, NG, WJ;
     int mode, layer;
+    int head_base;  // layer-wide index of query head 0 of this call (round-robin offset only)
     float c_log2;  // log2(e) / (S * sqrt(d))
 };
 
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParam
         if (rho < R) {
             const int h = h0 + rho / r;
             const long i = (long)I * r + rho % r;
-            const long pos = i * p.S + rr_offset(h, p.S, p.mode, p.layer);
+            const long pos = i * p.S + rr_offset(p.head_base + h, p.S, p.mode, p.layer);
             v = __ldg(reinterpret_cast<const uint4 *>(p.Q + ((long)h * p.L + pos) * D) + c);
         }
         *reinterpret_cast<uint4 *>(qs + rho * QSTRIDE + c * 8) = v;
@@ -332,7 +333,7 @@ bool estimate_supported(int H, int Hkv, int d, int S, int B, int L) {
 }
 
 rr_status_t launch_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, int d,
-                            int S, int B, int mode, int layer, float *A, void *ws,
+                            int S, int B, int mode, int layer, int head_base, float *A, void *ws,
                             cudaStream_t st) {
     const int Ns = L / S, Nb = L / B;
     EstPlan pl;
@@ -374,6 +375,7 @@ rr_status_t launch_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv
     p.WJ = pl.WJ;
     p.mode = mode;
     p.layer = layer;
+    p.head_base = head_base;
     p.c_log2 = (float)(1.4426950408889634 / ((double)S * sqrt((double)d)));
     dim3 grid(Nb, Hkv * pl.nHC);
     auto launch = [&](auto kern) -> rr_status_t {

@@ -5,21 +5,23 @@
 //
 // One CTA per (query head h, query block I): a 128-row query tile (for B = 64 the upper 64
 // rows are padding that is computed and never stored).  The CTA walks only the CSR entries
-// of row h*Nb + I.  Warp roles:
-//   warp 0      TMA producer: Q tile once, then K and V tiles of each selected block into a
-//               ring of 3-4 stages (128-byte swizzle, mbarrier transaction counts).
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T (both operands in shared memory) into
-//               one of two TMEM buffers, then O += P_j V_j with P_j read from TMEM (the
-//               A-from-tensor-memory form) and V_j from shared memory; completion is signalled
-//               by tcgen05.commit.
-//   warp 2      TMEM allocation / release.
-//   warps 4-7   softmax: one thread per query row (TMEM lane).  Online softmax in fp32 with a
+// of row h*Nb + I, each key block as 64-key sub-blocks.  Two CTAs share an SM, so each SM
+// sub-partition runs two independent softmax streams.  Warp roles (224 threads):
+//   warp 0      TMA producer of Q (once) and of the K sub-tiles, into a ring of two or more
+//               (128-byte swizzle, mbarrier transaction counts); L2 prefetch of upcoming
+//               sub-tiles; TMEM allocation / release.
+//   warp 1      TMA producer of the V sub-tiles (its own ring, so K loads never queue behind
+//               a V slot that is still being read).
+//   warp 2      MMA issuer (one thread): S_t = Q K_t^T (both operands in shared memory) into
+//               the single S buffer as soon as the softmax has loaded S_{t-1}, so S_t is
+//               computed while the softmax works on S_{t-1}; then O += P_t V_t with P_t read
+//               from TMEM (the A-from-tensor-memory form).  Completion is signalled by
+//               tcgen05.commit.
+//   warps 3-6   softmax: one thread per query row (TMEM lane).  Online softmax in fp32 with a
 //               lazily rescaled running max (O is rescaled in TMEM only when a row's max grows
-//               by more than 2^8), P packed to bf16 pairs and stored back into TMEM (two
-//               buffers, so block j's softmax never waits for block j-1's P*V), final
-//               normalisation and bf16 store of O.
-// TMEM columns: S0, S1 (fp32, B each), O (fp32, d), P0, P1 (bf16 pairs, B/2 each).
-// The producer also prefetches the K/V tiles of the next few selected blocks into L2.
+//               by more than 2^8), P packed to bf16 pairs and stored into one of two TMEM P
+//               buffers, final normalisation and bf16 store of O.
+// TMEM columns (256 per CTA): S [0, 64) fp32, P0 and P1 [64, 128) bf16 pairs, O [128, 128+d).
 // K and V come from KV head h / (H/Hkv); the heads of a KV group run as adjacent CTAs so
 // their K/V tiles are served from L2.  Every wait is bounded (about one second of
 // %globaltimer); a timeout sets a device error bit and the CTA drains and exits.
@@ -62,6 +64,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+
 // Packed pairs of fp32 (one 64-bit register, two lanes of the FMA pipe per instruction).
 typedef unsigned long long f32x2;
 __device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
@@ -84,53 +93,64 @@ __device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
 }
 
 constexpr int kBM = 128;  // query rows per CTA
+constexpr int kSub = 64;  // keys per sub-block: the unit of S, P and the K/V pipeline
 
 template <int D, int BN>
 struct TcCfg {
-    static constexpr int DC = D / 64;  // 64-element (128-byte) column chunks
+    static constexpr int DC = D / 64;       // 64-element (128-byte) column chunks
+    static constexpr int NSB = BN / kSub;   // sub-blocks per key block
     static constexpr uint32_t Q_BYTES = kBM * D * 2;
-    static constexpr uint32_t KV_BYTES = BN * D * 2;
-    // as many K/V stages (up to 4) as fit next to Q in the 227 KB a CTA may use (1024 bytes
-    // of alignment slack, 256 for barriers)
-    static constexpr int PF = 4;  // K/V blocks prefetched into L2 ahead of the shared-memory loads
-    static constexpr int NS_FIT = (int)((227u * 1024u - Q_BYTES - 1024u - 256u) / (2u * KV_BYTES));
-    static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
-    static constexpr uint32_t BAR_OFF = Q_BYTES + 2 * NS * KV_BYTES;
-    static constexpr uint32_t NBAR = 1 + 2 * NS + 2 + 1 + 1 + 1;
+    static constexpr uint32_t SUB_BYTES = kSub * D * 2;  // one K or V sub-tile
+    // Two CTAs per SM: each may use 113 KB of shared memory (1024 bytes of that are
+    // alignment slack, 256 barriers); the rest holds K and V sub-tile rings.
+    static constexpr int SLOTS = (int)((113u * 1024u - 1024u - 256u - Q_BYTES) / SUB_BYTES);
+    static constexpr int NK = SLOTS / 2 > 4 ? 4 : SLOTS / 2;
+    static constexpr int NV = NK;
+    static constexpr int PF = 8;  // sub-blocks prefetched into L2 ahead of the shared-memory loads
+    static constexpr uint32_t BAR_OFF = Q_BYTES + (NK + NV) * SUB_BYTES;
+    // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full, s_free, p_full[2],
+    // o_bar, fin
+    static constexpr uint32_t NBAR = 1 + 2 * NK + 2 * NV + 6;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
-    // TMEM columns: S0 [0,BN) S1 [BN,2BN) O [2BN,2BN+D) P0, P1 [2BN+D, 2BN+D+BN) (bf16 pairs,
-    // BN/2 columns each)
-    static constexpr uint32_t S_COL = 0, O_COL = 2 * BN, P_COL = 2 * BN + D;
-    static constexpr uint32_t TMEM_NEED = 2 * BN + D + BN;
-    static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
-    static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, BN, false);
+    // at least 80 KB so that a third CTA never fits on an SM (3 x 80 KB > 228 KB): with two
+    // CTAs of 256 TMEM columns each, a TMEM allocation never waits
+    static constexpr uint32_t SMEM_LAUNCH = SMEM + 1024 > 80u * 1024u ? SMEM + 1024 : 80u * 1024u;
+    // TMEM columns: S [0, 64) fp32 (one sub-block), P0 and P1 [64, 128) (bf16 pairs, 32 columns
+    // each), O [128, 128 + D) fp32
+    static constexpr uint32_t S_COL = 0, P_COL = kSub, O_COL = 2 * kSub;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, kSub, false);
     static constexpr uint32_t IDESC_PV = sm100::idesc_bf16(kBM, D, true);
-    static_assert(NS >= 2, "need at least two K/V stages");
-    static_assert(SMEM + 1024 <= 227u * 1024u, "shared memory budget");
-    static_assert(TMEM_NEED <= 512, "TMEM budget");
+    static_assert(BN % kSub == 0, "key blocks are whole sub-blocks");
+    static_assert(NK >= 2, "need at least two K and two V sub-tiles");
+    static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM + 1024 <= 113u * 1024u, "two CTAs per SM");
 };
 
 template <int D, int BN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(224, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, uint16_t *__restrict__ O,
                       const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
                       int H, int Hkv, int L, int Nb, float scale_log2) {
     using C = TcCfg<D, BN>;
-    constexpr int kNS = C::NS;
+    constexpr int NK = C::NK, NV = C::NV, NSB = C::NSB;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_u32(base);
     const uint32_t sK = sQ + C::Q_BYTES;
-    const uint32_t sV = sK + kNS * C::KV_BYTES;
+    const uint32_t sV = sK + NK * C::SUB_BYTES;
     const uint32_t sBar = sQ + C::BAR_OFF;
     const uint32_t q_full = sBar;
-    auto kv_full = [&](int s) { return sBar + 8u * (1 + s); };
-    auto kv_empty = [&](int s) { return sBar + 8u * (1 + kNS + s); };
-    auto s_full = [&](int b) { return sBar + 8u * (1 + 2 * kNS + b); };
-    const uint32_t p_full = sBar + 8u * (3 + 2 * kNS);
-    const uint32_t o_bar = sBar + 8u * (4 + 2 * kNS);
-    const uint32_t fin_bar = sBar + 8u * (5 + 2 * kNS);
+    auto k_full = [&](int s) { return sBar + 8u * (1 + s); };
+    auto k_empty = [&](int s) { return sBar + 8u * (1 + NK + s); };
+    auto v_full = [&](int s) { return sBar + 8u * (1 + 2 * NK + s); };
+    auto v_empty = [&](int s) { return sBar + 8u * (1 + 2 * NK + NV + s); };
+    const uint32_t s_full = sBar + 8u * (1 + 2 * NK + 2 * NV);
+    const uint32_t s_free = s_full + 8;
+    auto p_full = [&](int t) { return s_full + 16u + 8u * (t & 1); };
+    const uint32_t o_bar = s_full + 32;
+    const uint32_t fin_bar = s_full + 40;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + C::BAR_OFF + C::NBAR * 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,22 +165,27 @@ __global__ void __launch_bounds__(256, 1)
     const int h = g * G + within % G;
     const long crow = (long)h * Nb + I;
     const int e0 = row_ptr[crow];
-    const int n = row_ptr[crow + 1] - e0;
+    const int nsub = (row_ptr[crow + 1] - e0) * NSB;  // sub-block t: block e0 + t / NSB, half t % NSB
 
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 64) {
         sm100::mbar_init(q_full, 1);
-        for (int s = 0; s < kNS; ++s) {
-            sm100::mbar_init(kv_full(s), 1);
-            sm100::mbar_init(kv_empty(s), 1);
+        for (int s = 0; s < NK; ++s) {
+            sm100::mbar_init(k_full(s), 1);
+            sm100::mbar_init(k_empty(s), 1);
         }
-        sm100::mbar_init(s_full(0), 1);
-        sm100::mbar_init(s_full(1), 1);
-        sm100::mbar_init(p_full, 128);
+        for (int s = 0; s < NV; ++s) {
+            sm100::mbar_init(v_full(s), 1);
+            sm100::mbar_init(v_empty(s), 1);
+        }
+        sm100::mbar_init(s_full, 1);
+        sm100::mbar_init(s_free, 128);
+        sm100::mbar_init(p_full(0), 128);
+        sm100::mbar_init(p_full(1), 128);
         sm100::mbar_init(o_bar, 1);
         sm100::mbar_init(fin_bar, 1);
         sm100::fence_mbar_init();
     }
-    if (warp == 2) {
+    if (warp == 0) {
         sm100::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         sm100::tmem_relinquish();
     }
@@ -168,148 +193,198 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    auto key_row = [&](int t) { return g * L + __ldg(col_idx + e0 + t / NSB) * BN + (t % NSB) * kSub; };
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------------------------------------------------------- producer
+            // ------------------------------------------------------- K producer (and Q)
             sm100::prefetch_tmap(&tmQ);
             sm100::prefetch_tmap(&tmK);
             sm100::prefetch_tmap(&tmV);
             sm100::mbar_arrive_expect_tx(q_full, C::Q_BYTES);
             for (int c = 0; c < C::DC; ++c)
                 sm100::tma_load_2d(sQ + c * kBM * 128, &tmQ, c * 64, h * L + I * BN, q_full);
-            int issued = 0;
-            bool ok = true;
-            for (int j = 0; j < n && j < C::PF; ++j) {
-                const int Jp = __ldg(col_idx + e0 + j);
+            for (int t = 0; t < nsub && t < C::PF; ++t) {
+                const int y = key_row(t);
                 for (int c = 0; c < C::DC; ++c) {
-                    sm100::tma_prefetch_2d(&tmK, c * 64, g * L + Jp * BN);
-                    sm100::tma_prefetch_2d(&tmV, c * 64, g * L + Jp * BN);
+                    sm100::tma_prefetch_2d(&tmK, c * 64, y);
+                    sm100::tma_prefetch_2d(&tmV, c * 64, y);
                 }
             }
-            for (int j = 0; j < n; ++j) {
-                if (j + C::PF < n) {
-                    const int Jp = __ldg(col_idx + e0 + j + C::PF);
+            int issued = 0;
+            bool ok = true;
+            for (int t = 0; t < nsub; ++t) {
+                if (t + C::PF < nsub) {
+                    const int y = key_row(t + C::PF);
                     for (int c = 0; c < C::DC; ++c) {
-                        sm100::tma_prefetch_2d(&tmK, c * 64, g * L + Jp * BN);
-                        sm100::tma_prefetch_2d(&tmV, c * 64, g * L + Jp * BN);
+                        sm100::tma_prefetch_2d(&tmK, c * 64, y);
+                        sm100::tma_prefetch_2d(&tmV, c * 64, y);
                     }
                 }
-                const int s = j % kNS;
-                if (!wait_bar(kv_empty(s), ((j / kNS) & 1) ^ 1)) {
+                const int s = t % NK;
+                if (!wait_bar(k_empty(s), ((t / NK) & 1) ^ 1)) {  // S_{t-NK} has completed
                     ok = false;
                     break;
                 }
-                const int J = __ldg(col_idx + e0 + j);
-                sm100::mbar_arrive_expect_tx(kv_full(s), 2 * C::KV_BYTES);
-                for (int c = 0; c < C::DC; ++c) {
-                    sm100::tma_load_2d(sK + s * C::KV_BYTES + c * BN * 128, &tmK, c * 64, g * L + J * BN,
-                                       kv_full(s));
-                    sm100::tma_load_2d(sV + s * C::KV_BYTES + c * BN * 128, &tmV, c * 64, g * L + J * BN,
-                                       kv_full(s));
-                }
-                issued = j + 1;
+                const int y = key_row(t);
+                sm100::mbar_arrive_expect_tx(k_full(s), C::SUB_BYTES);
+                for (int c = 0; c < C::DC; ++c)
+                    sm100::tma_load_2d(sK + s * C::SUB_BYTES + c * kSub * 128, &tmK, c * 64, y, k_full(s));
+                issued = t + 1;
             }
             if (!ok) {
                 atomicOr(&g_device_errors, kErrTimeoutProducer);
                 // let the copies already in flight land before the CTA's memory is released
                 wait_bar(q_full, 0);
-                for (int j = issued > kNS ? issued - kNS : 0; j < issued; ++j)
-                    wait_bar(kv_full(j % kNS), (j / kNS) & 1);
+                for (int t = issued > NK ? issued - NK : 0; t < issued; ++t)
+                    wait_bar(k_full(t % NK), (t / NK) & 1);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            // ------------------------------------------------------------- V producer
+            int issued = 0;
+            bool ok = true;
+            for (int t = 0; t < nsub; ++t) {
+                const int s = t % NV;
+                if (!wait_bar(v_empty(s), ((t / NV) & 1) ^ 1)) {  // P_{t-NV} V_{t-NV} has completed
+                    ok = false;
+                    break;
+                }
+                const int y = key_row(t);
+                sm100::mbar_arrive_expect_tx(v_full(s), C::SUB_BYTES);
+                for (int c = 0; c < C::DC; ++c)
+                    sm100::tma_load_2d(sV + s * C::SUB_BYTES + c * kSub * 128, &tmV, c * 64, y, v_full(s));
+                issued = t + 1;
+            }
+            if (!ok) {
+                atomicOr(&g_device_errors, kErrTimeoutProducer);
+                for (int t = issued > NV ? issued - NV : 0; t < issued; ++t)
+                    wait_bar(v_full(t % NV), (t / NV) & 1);
+            }
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
             // ---------------------------------------------------------------- MMA issuer
             bool ok = wait_bar(q_full, 0);
             sm100::tc_fence_after();
-            auto issue_s = [&](int j) -> bool {
-                const int s = j % kNS, b = j & 1;
-                if (!wait_bar(kv_full(s), (j / kNS) & 1)) return false;
+            auto issue_s = [&](int t) -> bool {
+                const int s = t % NK;
+                if (!wait_bar(k_full(s), (t / NK) & 1)) return false;
                 sm100::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk >> 2, w = kk & 3;
                     const uint64_t ad = sm100::smem_desc_sw128(sQ + c * kBM * 128 + w * 32, 16, 1024);
                     const uint64_t bd =
-                        sm100::smem_desc_sw128(sK + s * C::KV_BYTES + c * BN * 128 + w * 32, 16, 1024);
-                    sm100::mma_ss(tmem + C::S_COL + b * BN, ad, bd, C::IDESC_S, kk > 0);
+                        sm100::smem_desc_sw128(sK + s * C::SUB_BYTES + c * kSub * 128 + w * 32, 16, 1024);
+                    sm100::mma_ss(tmem + C::S_COL, ad, bd, C::IDESC_S, kk > 0);
                 }
-                sm100::mma_commit(s_full(b));
+                sm100::mma_commit(k_empty(s));
+                sm100::mma_commit(s_full);
                 return true;
             };
-            if (ok && n > 0) ok = issue_s(0);
-            for (int j = 0; ok && j < n; ++j) {
-                if (j + 1 < n && !issue_s(j + 1)) {
+            if (ok && nsub > 0) ok = issue_s(0);
+            for (int t = 0; ok && t < nsub; ++t) {
+                // S_{t+1} goes into the S columns once every softmax thread has loaded S_t
+                if (t + 1 < nsub && !(wait_bar(s_free, t & 1) && issue_s(t + 1))) {
                     ok = false;
                     break;
                 }
-                if (!wait_bar(p_full, j & 1)) {
+                if (!wait_bar(p_full(t), (t >> 1) & 1) || !wait_bar(v_full(t % NV), (t / NV) & 1)) {
                     ok = false;
                     break;
                 }
                 sm100::tc_fence_after();
-                const int s = j % kNS;
+                const int s = t % NV;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
+                for (int kk = 0; kk < kSub / 16; ++kk) {
                     const uint64_t bd =
-                        sm100::smem_desc_sw128(sV + s * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024);
-                    sm100::mma_ts(tmem + C::O_COL, tmem + C::P_COL + (j & 1) * (BN / 2) + kk * 8, bd,
-                                  C::IDESC_PV, (j > 0 || kk > 0));
+                        sm100::smem_desc_sw128(sV + s * C::SUB_BYTES + kk * 16 * 128, kSub * 128, 1024);
+                    sm100::mma_ts(tmem + C::O_COL, tmem + C::P_COL + (t & 1) * (kSub / 2) + kk * 8, bd,
+                                  C::IDESC_PV, (t > 0 || kk > 0));
                 }
                 sm100::mma_commit(o_bar);
-                sm100::mma_commit(kv_empty(s));
+                sm100::mma_commit(v_empty(s));
             }
-            // every MMA issued must complete before the TMEM is released
+            // fin_bar: every MMA has completed (the epilogue reads O, then the TMEM is released)
             sm100::mma_commit(fin_bar);
             if (!wait_bar(fin_bar, 0)) ok = false;
             if (!ok) atomicOr(&g_device_errors, kErrTimeoutMma);
         }
-    } else if (warp >= 4) {
+    } else {
         // -------------------------------------------------------------------- softmax
-        const int r = threadIdx.x - 128;  // query row within the tile = TMEM lane
+        // warps 3-6; a warp may only touch TMEM lanes 32*(warp % 4) .. +31
+        const int r = (warp & 3) * 32 + lane;  // query row within the tile = TMEM lane
         const long qpos = (long)I * BN + r;
-        const uint32_t trow = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const int b = j & 1;
-            ok = __all_sync(0xffffffffu, wait_bar(s_full(b), (j >> 1) & 1));
+        for (int t = 0; t < nsub; ++t) {
+            ok = __all_sync(0xffffffffu, wait_bar(s_full, t & 1));
             if (!ok) break;
             sm100::tc_fence_after();
-            const int J = __ldg(col_idx + e0 + j);
-            uint32_t sr[BN];
-#pragma unroll
-            for (int cc = 0; cc < BN / 32; ++cc)
-                sm100::tmem_ld32(trow + C::S_COL + b * BN + cc * 32,
-                                 *reinterpret_cast<uint32_t(*)[32]>(sr + cc * 32));
+            uint32_t sr[kSub];
+            sm100::tmem_ld32(trow + C::S_COL, *reinterpret_cast<uint32_t(*)[32]>(sr));
+            sm100::tmem_ld32(trow + C::S_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
             sm100::tmem_wait_ld();
-            const bool diag = (J == I);
-            if (diag) {  // diagonal block: key i of the block is visible iff i <= r
+            // S_t is in registers: the MMA warp may write S_{t+1}
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(s_free);
+            const int J = __ldg(col_idx + e0 + t / NSB);
+            if (J == I) {  // diagonal block: key k0 + i of the block is visible iff k0 + i <= r
+                const int k0 = (t % NSB) * kSub;
 #pragma unroll
-                for (int i = 0; i < BN; ++i)
-                    if (i > r) sr[i] = __float_as_uint(-INFINITY);
+                for (int i = 0; i < kSub; ++i)
+                    if (k0 + i > r) sr[i] = __float_as_uint(-INFINITY);
             }
-            float mq[8];
+            // row max: four chains of three-input maxima
+            float mq[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mq[k] = __uint_as_float(sr[k]);
+            for (int k = 0; k < 4; ++k) mq[k] = __uint_as_float(sr[k]);
 #pragma unroll
-            for (int i = 8; i < BN; ++i) mq[i & 7] = fmaxf(mq[i & 7], __uint_as_float(sr[i]));
-            const float mraw = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
-                                     fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
-            const float mx = mraw * scale_log2;  // scale > 0 keeps the order
+            for (int i = 4; i + 8 <= kSub; i += 8)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mq[k] = fmax3(mq[k], __uint_as_float(sr[i + 2 * k]), __uint_as_float(sr[i + 2 * k + 1]));
+            mq[0] = fmax3(mq[0], __uint_as_float(sr[kSub - 4]), __uint_as_float(sr[kSub - 3]));
+            mq[1] = fmax3(mq[1], __uint_as_float(sr[kSub - 2]), __uint_as_float(sr[kSub - 1]));
+            const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * scale_log2;  // scale > 0
             // Lazy rescale: a row keeps its stale max while p <= 2^8.  The decision is per row,
-            // but tcgen05.ld/st are warp-collective, so the O rescale runs for the whole warp
-            // whenever any of its rows needs it (alpha = 1 on the others).  Only then must the
-            // previous block's P*V be complete; P itself is double-buffered.
+            // but tcgen05.ld/st are warp-collective, so the O rescale (after the exponentials,
+            // below) runs for the whole warp whenever any of its rows needs it (alpha = 1 on
+            // the others), once P_{t-1} V_{t-1} is complete.
             const bool need = mx > m + 8.f;
             float alpha = 1.f;
             if (need) {
-                alpha = ex2_approx(m - mx);  // 0 on a row's first block
+                alpha = ex2_approx(m - mx);  // 0 on a row's first sub-block
                 l *= alpha;
+                m = mx;
             }
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                ok = __all_sync(0xffffffffu, wait_bar(o_bar, (j - 1) & 1));
+            // P_t goes to the buffer P_{t-2} used.  Its P*V product is complete: S_t was issued
+            // after P_{t-2} V_{t-2}, and the commit behind S_t (waited for above) fires only
+            // once every earlier MMA of the issuing thread is done.
+            const float nm = (m == -INFINITY) ? 0.f : -m;  // a row with nothing attended yet
+            const f32x2 sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(nm, nm);
+            f32x2 rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+            uint32_t pk[kSub / 2];
+#pragma unroll
+            for (int e = 0; e < kSub / 2; ++e) {
+                const f32x2 x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                        sc2, nm2);
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                rs2[e & 1] = f2_add(rs2[e & 1], f2_pack(p0, p1));
+                pk[e] = pack_bf16(p0, p1);
+            }
+            sm100::tmem_st32(trow + C::P_COL + (t & 1) * (kSub / 2), pk);
+            float ra, rb, rc, rd;
+            f2_unpack(rs2[0], ra, rb);
+            f2_unpack(rs2[1], rc, rd);
+            l += (ra + rb) + (rc + rd);
+            if (t > 0 && __any_sync(0xffffffffu, need)) {
+                ok = __all_sync(0xffffffffu, wait_bar(o_bar, (t - 1) & 1));
                 if (!ok) break;
                 sm100::tc_fence_after();
 #pragma unroll
@@ -322,52 +397,34 @@ __global__ void __launch_bounds__(256, 1)
                     sm100::tmem_st32(trow + C::O_COL + cc * 32, rg);
                 }
             }
-            if (need) m = mx;
-            // P_j goes to the buffer P_{j-2} used.  Its P*V product is complete: S_j was issued
-            // after P_{j-2} V_{j-2}, and the commit behind S_j (which this warpgroup waited for
-            // before reading S_j) fires only once every earlier MMA of the issuing thread is done.
-            const float nm = (m == -INFINITY) ? 0.f : -m;  // a row with nothing attended yet
-            const f32x2 sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(nm, nm);
-            f32x2 rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-#pragma unroll
-            for (int hc = 0; hc < BN / 64; ++hc) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const f32x2 x2 = f2_fma(f2_pack(__uint_as_float(sr[hc * 64 + 2 * e]),
-                                                    __uint_as_float(sr[hc * 64 + 2 * e + 1])),
-                                            sc2, nm2);
-                    float x0, x1;
-                    f2_unpack(x2, x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    rs2[e & 1] = f2_add(rs2[e & 1], f2_pack(p0, p1));
-                    pk[e] = pack_bf16(p0, p1);
-                }
-                sm100::tmem_st32(trow + C::P_COL + (j & 1) * (BN / 2) + hc * 32, pk);
-            }
-            float ra, rb, rc, rd;
-            f2_unpack(rs2[0], ra, rb);
-            f2_unpack(rs2[1], rc, rd);
-            const float rs = (ra + rb) + (rc + rd);
             sm100::tmem_wait_st();
-            l += rs;
             sm100::tc_fence_before();
-            sm100::mbar_arrive(p_full);
+            sm100::mbar_arrive(p_full(t));
         }
-        if (ok && n > 0) {
-            ok = __all_sync(0xffffffffu, wait_bar(o_bar, (n - 1) & 1));
+        // O is final once every MMA has completed.  (o_bar cannot say so: when the last
+        // softmax step ends, only the P*V of two steps earlier is known to be complete, so the
+        // barrier may still be two phases short and a parity wait on it would alias.)
+        if (ok) {
+            ok = __all_sync(0xffffffffu, wait_bar(fin_bar, 0));
             sm100::tc_fence_after();
         }
         if (!ok) {
             if (lane == 0) atomicOr(&g_device_errors, kErrTimeoutSoftmax);
         } else {
+            // a row that attended nothing (an empty CSR row) is written as zeros: its O columns
+            // in TMEM were never written
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             uint16_t *orow = O + ((long)h * L + qpos) * D;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t rg[32];
-                sm100::tmem_ld32(trow + C::O_COL + cc * 32, rg);
-                sm100::tmem_wait_ld();
+                if (nsub > 0) {
+                    sm100::tmem_ld32(trow + C::O_COL + cc * 32, rg);
+                    sm100::tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) rg[i] = 0u;
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -383,7 +440,8 @@ __global__ void __launch_bounds__(256, 1)
     }
     sm100::tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 0) {
+        __syncwarp();  // lane 0 ran the producer; dealloc is warp-collective
         sm100::tc_fence_after();
         sm100::tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -427,19 +485,17 @@ rr_status_t launch_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, i
                       cudaStream_t st) {
     using C = TcCfg<D, BN>;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, Q, (uint64_t)H * L, D, kBM) || !make_map(&mk, K, (uint64_t)Hkv * L, D, BN) ||
-        !make_map(&mv, V, (uint64_t)Hkv * L, D, BN))
+    if (!make_map(&mq, Q, (uint64_t)H * L, D, kBM) || !make_map(&mk, K, (uint64_t)Hkv * L, D, kSub) ||
+        !make_map(&mv, V, (uint64_t)Hkv * L, D, kSub))
         return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cuTensorMapEncodeTiled failed");
-    // at least 116 KB of shared memory: one CTA per SM, so TMEM allocation never contends
-    size_t smem = C::SMEM + 1024;
-    if (smem < 116 * 1024) smem = 116 * 1024;
+    const size_t smem = C::SMEM_LAUNCH;
     auto kern = prefill_tc_kernel<D, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     const int Nb = L / BN;
     dim3 grid((unsigned)((long)H * Nb));
-    kern<<<grid, 256, smem, st>>>(mq, mk, mv, O, row_ptr, col_idx, H, Hkv, L, Nb,
+    kern<<<grid, 224, smem, st>>>(mq, mk, mv, O, row_ptr, col_idx, H, Hkv, L, Nb,
                                   scale * 1.4426950408889634f);
     return check_launch("rr_sparse_prefill: prefill_tc_kernel");
 }

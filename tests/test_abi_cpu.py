@@ -77,6 +77,29 @@ def test_estimate_rejections(L):
     assert _est(L, Len=0, q=0, k=0, out=0, ws=0) == 0   # empty problem: accepted, no launch
 
 
+def test_estimate_heads_rejections(L):
+    f = L.rr_estimate_heads
+    ok = (FAKE, FAKE, 4, 2, 256, 64, 8, 64, 0, 0)
+    assert f(*ok, -1, FAKE, FAKE, 1 << 30, None) == INVALID
+    assert f(*ok, (1 << 20) + 1, FAKE, FAKE, 1 << 30, None) == INVALID
+    assert b"head_base" in L.rr_last_error()
+    assert f(FAKE, FAKE, 4, 2, 0, 64, 8, 64, 0, 0, 4, 0, 0, 0, None) == 0   # empty: no launch
+
+
+def test_host_path_argument_checks(L):
+    import torch
+
+    Q = torch.zeros(4, 128, 64, dtype=torch.bfloat16)
+    K = torch.zeros(2, 128, 64, dtype=torch.bfloat16)
+    assert rr.default_chunks(8) == 8 and rr.default_chunks(28) == 7 and rr.default_chunks(1) == 1
+    with pytest.raises(rr.RRAttnError, match="chunks=3"):
+        rr.prefill(Q, K, K, 8, 64, 0.9, chunks=3)
+    with pytest.raises(rr.RRAttnError, match="shapes"):
+        rr.prefill(Q, K[:, :64].contiguous(), K, 8, 64, 0.9)
+    with pytest.raises(rr.RRAttnError, match="contiguous bf16"):
+        rr.prefill(Q.float(), K, K, 8, 64, 0.9)
+
+
 def test_select_rejections(L):
     P = FAKE
     ok_cap = 2 * 4 * 5 // 2

@@ -228,15 +228,39 @@ def test_validate_csr_counts_corruption(cuda_device):
     assert rr.validate_csr(torch.from_numpy(rp2).cuda(), cig, H, Nb) >= 1
 
 
-def test_host_tensors_through_public_api(cuda_device):
-    w = workloads.get(1, H=8, Hkv=2, L=2048)
+@pytest.mark.parametrize("chunks", [None, 1, 4])
+def test_host_tensors_through_public_api(chunks, cuda_device):
+    # host path: slices of KV groups copied in / computed / copied back on three streams;
+    # identical bytes to the one-pass device call (heads 4.. of a slice keep their offsets)
+    w = workloads.get(1, H=16, Hkv=4, L=2048)
     t = workloads.generate(w)
     pinned = {k: v.pin_memory() for k, v in t.items()}
-    O_host = rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau)
+    O_host = rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, chunks=chunks)
     assert not O_host.is_cuda
     d = _to(t, cuda_device)
     O_dev = rr.prefill(d["Q"], d["K"], d["V"], w.S, w.B, w.tau)
     assert torch.equal(O_host.view(torch.int16), O_dev.cpu().view(torch.int16))
+    assert rr.device_errors() == 0
+
+
+@pytest.mark.parametrize("strategy,layer", [("head", 0), ("hybrid", 3), ("layer", 2), ("none", 0)])
+def test_estimate_head_slices(strategy, layer, cuda_device):
+    # a slice of whole KV groups estimated with its layer-wide head index equals the
+    # matching rows of the whole layer's estimate, bit for bit, and the oracle's rows
+    w = workloads.get(1, H=8, Hkv=4, L=2048)
+    G = w.H // w.Hkv
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    A = rr.estimate(d["Q"], d["K"], w.S, w.B, strategy=strategy, layer=layer)
+    for g0, g1 in [(0, 1), (1, 3), (3, 4), (0, 4)]:
+        As = rr.estimate(d["Q"][g0 * G:g1 * G], d["K"][g0:g1], w.S, w.B, strategy=strategy,
+                         layer=layer, head_base=g0 * G)
+        assert torch.equal(As, A[g0 * G:g1 * G]), (g0, g1)
+    mode = {"head": oracle.HEAD_RR, "none": oracle.NO_RR, "layer": oracle.LAYER_RR,
+            "hybrid": oracle.HYBRID_RR}[strategy]
+    As = rr.estimate(d["Q"][2:6], d["K"][1:3], w.S, w.B, strategy=strategy, layer=layer, head_base=2)
+    A_or = oracle.estimate(t["Q"], t["K"], w.S, w.B, mode=mode, layer=layer, heads=(2, 6))
+    assert np.abs(As.cpu().numpy() - A_or[2:6]).max() <= SCORE_TOL
 
 
 FULL = [(i, workloads.get(i)) for i in (1, 2, 3, 4)]
