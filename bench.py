@@ -219,10 +219,17 @@ def run_reference(args):
     return 0
 
 
-def config_dict(w, world):
+def config_dict(w, world, shard="replicas"):
+    if world == 1:
+        par = "single"
+    elif shard == "heads":
+        par = f"heads{world} (KV groups split across ranks, no data-path collective)"
+    else:
+        par = f"replicas{world}"
     return {"workload": w.name, "H": w.H, "Hkv": w.Hkv, "L": w.L, "d": w.d, "S": w.S, "B": w.B,
-            "tau": w.tau, "recipe": w.recipe, "global_batch": world, "seq_len": w.L,
-            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "tau": w.tau, "recipe": w.recipe,
+            "global_batch": world if shard == "replicas" else 1, "seq_len": w.L,
+            "parallelism": par,
             "l2": "inputs larger than L2 (Q+K+V %.2f GB > 126 MB); no flush" %
                   (2 * w.L * w.d * (w.H + 2 * w.Hkv) / 1e9)}
 
@@ -254,17 +261,28 @@ def run_ours(args):
     w = workloads.get(args.workload)
     if args.L:
         w = w.with_(L=args.L)
-    host = workloads.generate(w, seed=rank)
+    if args.shard == "heads":
+        # one layer split by whole KV groups: every rank holds the same layer and computes
+        # its query heads [h0, h1) with their layer-wide round-robin offsets (strong scaling)
+        full = workloads.generate(w, seed=0)
+        h0, h1, g0, g1 = rr.head_shard(rank, world, w.H, w.Hkv)
+        host = {"Q": full["Q"][h0:h1].contiguous(), "K": full["K"][g0:g1].contiguous(),
+                "V": full["V"][g0:g1].contiguous()}
+        wl = w.with_(H=h1 - h0, Hkv=g1 - g0)
+    else:
+        # one independent layer per rank (weak scaling)
+        full = host = workloads.generate(w, seed=rank)
+        h0, wl = 0, w
     d = {k: v.to(dev) for k, v in host.items()}
     Q, K, V = d["Q"], d["K"], d["V"]
-    ws = rr.Workspace(w.H, w.Hkv, w.L, w.d, w.S, w.B, device=dev)
+    ws = rr.Workspace(wl.H, wl.Hkv, wl.L, wl.d, wl.S, wl.B, device=dev)
     O = torch.empty_like(Q)
     st = torch.cuda.current_stream(dev)
 
     def step(ev=None, tau=None):
         if ev:
             ev[0].record(st)
-        rr.estimate(Q, K, w.S, w.B, out=ws.block_scores, workspace=ws.est)
+        rr.estimate(Q, K, w.S, w.B, out=ws.block_scores, workspace=ws.est, head_base=h0)
         if ev:
             ev[1].record(st)
         rr.select(ws.block_scores, w.tau if tau is None else tau, True, row_ptr=ws.row_ptr,
@@ -304,25 +322,29 @@ def run_ours(args):
     rp = ws.row_ptr.cpu().numpy()
     nnz = int(rp[-1])
     ci = ws.col_idx[:nnz].cpu().numpy()
-    sel_flops, n_diag, n_off = selected_flops(rp, ci, w.H, w.Nb, w.B, w.d)
-    causal_blocks = w.H * w.Nb * (w.Nb + 1) // 2
+    sel_flops, n_diag, n_off = selected_flops(rp, ci, wl.H, wl.Nb, wl.B, wl.d)
+    causal_blocks = wl.H * wl.Nb * (wl.Nb + 1) // 2
     dense = dense_causal_flops(w)
+    # whole-job throughput: weak scaling processes one layer per rank, head sharding one
+    # layer in all
+    layers = world if args.shard == "replicas" else 1
     peaks, peak_kind = load_peaks()
     prefill_tflops = sel_flops / (stage["prefill_ms"] * 1e-3) / 1e12
-    est_bytes = (2 * w.Hkv * w.L * w.d              # K read
-                 + 2 * w.H * w.Ns * w.d             # sampled Q rows
-                 + 4 * w.Hkv * w.Ns * w.d * 2       # pooled keys written + read
-                 + 4 * w.H * w.Nb * w.Nb)           # block scores written
-    sel_bytes = 4 * w.H * w.Nb * w.Nb + 4 * (w.H * w.Nb + 1) + 4 * nnz
+    est_bytes = (2 * wl.Hkv * wl.L * wl.d           # K read
+                 + 2 * wl.H * wl.Ns * wl.d          # sampled Q rows
+                 + 4 * wl.Hkv * wl.Ns * wl.d * 2    # pooled keys written + read
+                 + 4 * wl.H * wl.Nb * wl.Nb)        # block scores written
+    sel_bytes = 4 * wl.H * wl.Nb * wl.Nb + 4 * (wl.H * wl.Nb + 1) + 4 * nnz
     line = {
         "metric": METRIC,
-        "value": aggregate_tflops(world, dense, ms_step),
+        "value": aggregate_tflops(layers, dense, ms_step),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "ms_per_layer": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "weak" if args.shard == "replicas" else "strong",
+        "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded generator, no datasets or weights)",
-        "config": config_dict(w, world),
+        "config": config_dict(w, world, args.shard),
         "stages": {**stage,
                    "estimate_gbs": est_bytes / (stage["estimate_ms"] * 1e-3) / 1e9,
                    "select_gbs": sel_bytes / (stage["select_ms"] * 1e-3) / 1e9,
@@ -336,18 +358,18 @@ def run_ours(args):
                      "frac_of_burst": prefill_tflops / peaks["bf16_tflops"],
                      "peak_source": f"{peak_kind} bf16 (sustained)",
                      "flops_per_launch": sel_flops,
-                     "traffic": prefill_traffic_per_launch(w),
+                     "traffic": prefill_traffic_per_launch(wl),
                      "traffic_unit": "bytes/launch (ncu dram read+write at L=32768, scaled by L)"},
         "gpu_launches": 6 * args.steps,
         "clocks": clocks,
     }
     # ---- extra measurements (outside the timed region)
     if rank == 0 and not args.quick:
-        line["tau_sweep"] = tau_sweep(w, step, st, ws, torch)
-        line["dense_reference"] = dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_step)
-    line["e2e"] = e2e(w, host, rr, torch, dev, args)
+        line["tau_sweep"] = tau_sweep(wl, step, st, ws, torch)
+        line["dense_reference"] = dense_comparison(wl, Q, K, V, ws, rr, torch, st, ms_step)
+    line["e2e"] = e2e(w, wl, host, h0, layers, rr, torch, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
-        layer_s, info = oracle_sample(w, host, n_rows=args.cpu_rows, n_est_heads=args.cpu_heads)
+        layer_s, info = oracle_sample(w, full, n_rows=args.cpu_rows, n_est_heads=args.cpu_heads)
         import oracle
 
         line["cpu_baseline"] = {
@@ -421,31 +443,31 @@ def dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_sparse):
     return res
 
 
-def e2e(w, host, rr, torch, dev, args):
-    """Same layer through the public API from pinned host buffers: H2D of Q/K/V, the three
-    stages, D2H of O, every step inside the timed region (the API overlaps the copies of one
-    slice of KV groups with the compute of another)."""
+def e2e(w, wl, host, h0, layers, rr, torch, dev, args):
+    """The rank's part of the job through the public API from pinned host buffers: H2D of
+    Q/K/V, the three stages, D2H of O, every step inside the timed region (the API overlaps
+    the copies of one slice of KV groups with the compute of another)."""
     pinned = {k: v.pin_memory() for k, v in host.items()}
     out = torch.empty(pinned["Q"].shape, dtype=torch.bfloat16, pin_memory=True)
-    ws = rr.Workspace(w.H, w.Hkv, w.L, w.d, w.S, w.B, device=dev)
     st = torch.cuda.current_stream(dev)
+    run = lambda: rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, out=out,
+                             head_base=h0)
     for _ in range(max(1, min(args.warmup, 2))):
-        rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, ws=ws, out=out)
+        run()
     n = max(1, min(args.steps, 5))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
     for _ in range(n):
-        rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, ws=ws, out=out)
+        run()
     e1.record(st)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / n, dev)
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    return {"value": aggregate_tflops(world, dense_causal_flops(w), ms), "unit": "TFLOP/s",
+    return {"value": aggregate_tflops(layers, dense_causal_flops(w), ms), "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n,
-            "pipeline": f"{rr.default_chunks(w.Hkv)} slices of whole KV groups; copy-in, compute "
+            "pipeline": f"{rr.default_chunks(wl.Hkv)} slices of whole KV groups; copy-in, compute "
                         f"and copy-out on three streams"}
 
 
@@ -462,6 +484,9 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=8192)
     ap.add_argument("--cpu-heads", type=int, default=4)
     ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="replicas: one independent layer per GPU (weak scaling); heads: one "
+                         "layer split across the GPUs by whole KV groups (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -22,7 +22,8 @@ import torch
 
 __all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
            "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
-           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors", "default_chunks"]
+           "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors", "default_chunks",
+           "head_shard"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "librrattn.so")
@@ -211,7 +212,7 @@ def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, t
             protect_last: bool = True, strategy: str = "head", layer: int = 0,
             scale: Optional[float] = None, ws: Optional[Workspace] = None,
             out: Optional[torch.Tensor] = None, return_intermediates: bool = False,
-            chunks: Optional[int] = None):
+            chunks: Optional[int] = None, head_base: int = 0):
     """One attention layer's sparse prefill: estimate -> select -> sparse attention.
 
     Host (CPU) tensors are accepted: the layer is then processed in `chunks` slices of whole
@@ -221,11 +222,14 @@ def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, t
     the copies asynchronous.  The result is identical to the one-pass device call: every
     stage is independent per query head, and each slice is estimated with its layer-wide
     head index.  The host path allocates its own slice-sized workspace (`ws` applies to the
-    device path); with return_intermediates it runs as one slice."""
+    device path); with return_intermediates it runs as one slice.
+
+    Q, K, V may themselves be a shard of whole KV groups of a larger layer (see head_shard);
+    head_base is then the layer-wide index of Q's first head."""
     host = not Q.is_cuda
     if host and not return_intermediates:
         return _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, scale,
-                                       out, chunks)
+                                       out, chunks, head_base)
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
         Q, K, V = (t.to(dev, non_blocking=True) for t in (Q, K, V))
@@ -233,7 +237,8 @@ def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, t
     Hkv = K.shape[0]
     if ws is None:
         ws = Workspace(H, Hkv, L, d, S, B, device=Q.device)
-    estimate(Q, K, S, B, strategy=strategy, layer=layer, out=ws.block_scores, workspace=ws.est)
+    estimate(Q, K, S, B, strategy=strategy, layer=layer, out=ws.block_scores, workspace=ws.est,
+             head_base=head_base)
     select(ws.block_scores, tau, protect_last, row_ptr=ws.row_ptr, col_idx=ws.col_idx,
            nnz=ws.nnz, workspace=ws.sel)
     O = sparse_prefill(Q, K, V, ws.row_ptr, ws.col_idx, B, scale=scale,
@@ -248,12 +253,29 @@ def prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, S: int, B: int, t
     return O
 
 
+def head_shard(rank: int, world: int, H: int, Hkv: int) -> Tuple[int, int, int, int]:
+    """Rank `rank`'s share of a layer split across `world` GPUs by whole KV groups:
+    (h0, h1, g0, g1) = its query heads [h0, h1) and KV heads [g0, g1), contiguous, with the
+    groups spread as evenly as they divide.  Every stage is independent per query head, so
+    the shards need no exchange; pass h0 as head_base to keep the round-robin offsets."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside world {world}")
+    if Hkv <= 0 or H % Hkv:
+        raise ValueError(f"H={H} is not a multiple of Hkv={Hkv}")
+    if world > Hkv:
+        raise ValueError(f"{world} ranks cannot share {Hkv} KV groups")
+    G = H // Hkv
+    g0, g1 = rank * Hkv // world, (rank + 1) * Hkv // world
+    return g0 * G, g1 * G, g0, g1
+
+
 def default_chunks(Hkv: int) -> int:
     """Slices of the host pipeline: the largest divisor of Hkv that is at most 8."""
     return max(c for c in range(1, min(Hkv, 8) + 1) if Hkv % c == 0)
 
 
-def _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, scale, out, chunks):
+def _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, scale, out, chunks,
+                            head_base=0):
     for n, t in (("Q", Q), ("K", K), ("V", V)):
         if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
             raise RRAttnError("prefill", 1, f"{n}: host path needs contiguous bf16 CPU tensors")
@@ -291,7 +313,7 @@ def _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, s
         hs, gs = slice(c * hc, (c + 1) * hc), slice(c * gc, (c + 1) * gc)
         compute.wait_event(loaded[c])
         estimate(Qd[hs], Kd[gs], S, B, strategy=strategy, layer=layer, out=ws.block_scores,
-                 workspace=ws.est, head_base=c * hc)
+                 workspace=ws.est, head_base=head_base + c * hc)
         select(ws.block_scores, tau, protect_last, row_ptr=ws.row_ptr, col_idx=ws.col_idx,
                nnz=ws.nnz, workspace=ws.sel)
         sparse_prefill(Qd[hs], Kd[gs], Vd[gs], ws.row_ptr, ws.col_idx, B, scale=scale, out=Od[hs])

@@ -243,6 +243,25 @@ def test_host_tensors_through_public_api(chunks, cuda_device):
     assert rr.device_errors() == 0
 
 
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_sharded_layer_equals_one_pass(world, cuda_device):
+    # the shards of a head-sharded layer (computed one after another here, each on its own)
+    # reproduce the one-pass layer byte for byte, through the device and the host paths
+    w = workloads.get(1, H=16, Hkv=4, L=2048)
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    O_ref = rr.prefill(d["Q"], d["K"], d["V"], w.S, w.B, w.tau)
+    for rank in range(world):
+        h0, h1, g0, g1 = rr.head_shard(rank, world, w.H, w.Hkv)
+        Qs, Ks, Vs = d["Q"][h0:h1].contiguous(), d["K"][g0:g1].contiguous(), d["V"][g0:g1].contiguous()
+        O_dev = rr.prefill(Qs, Ks, Vs, w.S, w.B, w.tau, head_base=h0)
+        assert torch.equal(O_dev, O_ref[h0:h1]), rank
+        host = [x.cpu().pin_memory() for x in (Qs, Ks, Vs)]
+        O_host = rr.prefill(*host, w.S, w.B, w.tau, head_base=h0)
+        assert torch.equal(O_host, O_ref[h0:h1].cpu()), rank
+    assert rr.device_errors() == 0
+
+
 @pytest.mark.parametrize("strategy,layer", [("head", 0), ("hybrid", 3), ("layer", 2), ("none", 0)])
 def test_estimate_head_slices(strategy, layer, cuda_device):
     # a slice of whole KV groups estimated with its layer-wide head index equals the
