@@ -222,11 +222,11 @@ __global__ void __launch_bounds__(224, 2)
                     }
                 }
                 const int s = t % NK;
+                const int y = key_row(t);
                 if (!wait_bar(k_empty(s), ((t / NK) & 1) ^ 1)) {  // S_{t-NK} has completed
                     ok = false;
                     break;
                 }
-                const int y = key_row(t);
                 sm100::mbar_arrive_expect_tx(k_full(s), C::SUB_BYTES);
                 for (int c = 0; c < C::DC; ++c)
                     sm100::tma_load_2d(sK + s * C::SUB_BYTES + c * kSub * 128, &tmK, c * 64, y, k_full(s));
@@ -247,11 +247,11 @@ __global__ void __launch_bounds__(224, 2)
             bool ok = true;
             for (int t = 0; t < nsub; ++t) {
                 const int s = t % NV;
+                const int y = key_row(t);
                 if (!wait_bar(v_empty(s), ((t / NV) & 1) ^ 1)) {  // P_{t-NV} V_{t-NV} has completed
                     ok = false;
                     break;
                 }
-                const int y = key_row(t);
                 sm100::mbar_arrive_expect_tx(v_full(s), C::SUB_BYTES);
                 for (int c = 0; c < C::DC; ++c)
                     sm100::tma_load_2d(sV + s * C::SUB_BYTES + c * kSub * 128, &tmV, c * 64, y, v_full(s));
@@ -320,6 +320,8 @@ __global__ void __launch_bounds__(224, 2)
         const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float m = -INFINITY, l = 0.f;
         bool ok = true;
+        // A CSR row is ascending with J <= I, so only its last block can be the diagonal one.
+        const int tdiag = (nsub > 0 && __ldg(col_idx + e0 + nsub / NSB - 1) == I) ? nsub - NSB : nsub;
         for (int t = 0; t < nsub; ++t) {
             ok = __all_sync(0xffffffffu, wait_bar(s_full, t & 1));
             if (!ok) break;
@@ -331,9 +333,8 @@ __global__ void __launch_bounds__(224, 2)
             // S_t is in registers: the MMA warp may write S_{t+1}
             sm100::tc_fence_before();
             sm100::mbar_arrive(s_free);
-            const int J = __ldg(col_idx + e0 + t / NSB);
-            if (J == I) {  // diagonal block: key k0 + i of the block is visible iff k0 + i <= r
-                const int k0 = (t % NSB) * kSub;
+            if (t >= tdiag) {  // diagonal block: key k0 + i of the block is visible iff k0 + i <= r
+                const int k0 = (t - tdiag) * kSub;
 #pragma unroll
                 for (int i = 0; i < kSub; ++i)
                     if (k0 + i > r) sr[i] = __float_as_uint(-INFINITY);
