@@ -97,7 +97,7 @@ __device__ __forceinline__ int rr_offset(int h, int S, int mode, int layer) {
 }
 
 template <int D, int MTW, int BPT>
-__global__ void __launch_bounds__(kEstThreads, 1) estimate_kernel(const EstParams p) {
+__global__ void __launch_bounds__(kEstThreads, MTW == 1 ? 2 : 1) estimate_kernel(const EstParams p) {
     constexpr int KS = D / 16;
     constexpr int QSTRIDE = D + 8;  // bf16 elements per staged query row (16-byte pad)
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -304,18 +304,22 @@ size_t est_smem(int R, int MT, int WJ, int Nb, int d) {
 
 bool plan_estimate(int H, int Hkv, int d, int S, int B, int Nb, EstPlan *pl) {
     const int G = H / Hkv, r = B / S;
-    for (int hc = G; hc >= 1; --hc) {
-        if (G % hc) continue;
-        const int R = hc * r;
-        if (R > 128) continue;
-        int MT = 1;
-        while (MT * 16 < R) MT *= 2;
-        const int MTW = MT < 2 ? MT : 2;
-        const int NG = MT / MTW, WJ = kEstWarps / NG;
-        const size_t sm = est_smem(R, MT, WJ, Nb, d);
-        if (sm > 200 * 1024) continue;
-        *pl = EstPlan{hc, G / hc, R, MT, MTW, NG, WJ, sm};
-        return true;
+    // Rows per CTA: exactly 16 (one m16 tile per warp, two CTAs per SM) when a whole number
+    // of heads gives 16 and it fits, else the largest chunk that fits (one CTA per SM).
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int hc = G; hc >= 1; --hc) {
+            if (G % hc) continue;
+            const int R = hc * r;
+            if (R > 128 || (pass == 0 && R != 16)) continue;
+            int MT = 1;
+            while (MT * 16 < R) MT *= 2;
+            const int MTW = MT < 2 ? MT : 2;
+            const int NG = MT / MTW, WJ = kEstWarps / NG;
+            const size_t sm = est_smem(R, MT, WJ, Nb, d);
+            if (sm > 200 * 1024) continue;
+            *pl = EstPlan{hc, G / hc, R, MT, MTW, NG, WJ, sm};
+            return true;
+        }
     }
     return false;
 }
