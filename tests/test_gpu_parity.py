@@ -214,6 +214,33 @@ def test_empty_sequence(cuda_device):
     assert O.shape == Q.shape
 
 
+@pytest.mark.parametrize("B,d", [(128, 128), (64, 64)])
+def test_empty_csr_rows_give_zero_output(B, d, cuda_device):
+    # a CSR row with no blocks attends to nothing: its output rows are exactly zero, and the
+    # other rows are unaffected (compared with the oracle under the same CSR)
+    w = workloads.get(0, H=4, Hkv=2, L=8 * B, d=d, S=8, B=B)
+    t = workloads.generate(w)
+    rp, ci = oracle.full_csr(w.H, w.Nb)
+    rows = _csr_rows(rp, ci)
+    empty = {3, 9, 17, 30}                       # (h, I) rows h*Nb + I
+    rows = [[] if r in empty else lst for r, lst in enumerate(rows)]
+    rp2 = np.concatenate([[0], np.cumsum([len(x) for x in rows])]).astype(np.int32)
+    ci2 = np.concatenate([np.asarray(x, np.int32) for x in rows if x]).astype(np.int32)
+    d_ = _to(t, cuda_device)
+    O = rr.sparse_prefill(d_["Q"], d_["K"], d_["V"], torch.from_numpy(rp2).cuda(),
+                          torch.from_numpy(ci2).cuda(), B)
+    torch.cuda.synchronize()
+    assert rr.device_errors() == 0
+    Oh = O.float().cpu().numpy()
+    for r in empty:
+        h, I = divmod(r, w.Nb)
+        assert not Oh[h, I * B:(I + 1) * B].any(), r
+    check = [(h, q) for h in range(w.H) for q in range(0, w.L, 7) if h * w.Nb + q // B not in empty]
+    O_ref = oracle.prefill_rows(t["Q"], t["K"], t["V"], B, rp2, ci2, check)
+    idx = torch.as_tensor(check)
+    _check_output(O.float().cpu()[idx[:, 0], idx[:, 1]].numpy(), O_ref)
+
+
 def test_validate_csr_counts_corruption(cuda_device):
     H, Nb = 2, 8
     rp, ci = oracle.full_csr(H, Nb)
