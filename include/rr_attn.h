@@ -23,10 +23,10 @@
  *   - L = 0 is accepted by every call as an empty problem: nothing is launched.
  *   - Supported: d in {64, 128}; B in {64, 128}; 1 <= S <= B with B % S == 0 and B/S = 4
  *     or a multiple of 8; (L/S) % 8 == 0; L % B == 0; H % Hkv == 0; L <= 2^20; H <= 256.
- *     rr_estimate also keeps, per CTA, the block sums of its sampled rows for a whole row of
- *     key blocks in shared memory (at least (B/S) * (L/B) * 4 bytes, under about 200 KB): at
- *     B/S = 8 that allows L/B <= 6216 (L <= 795,648 at B = 128).  Longer layers return
- *     RR_ERR_UNSUPPORTED from rr_estimate; rr_select and rr_sparse_prefill take L up to 2^20.
+ *     For B/S = 64 or 128 (S = 1, the exact mode) rr_estimate keeps, per CTA, the block sums
+ *     of its sampled rows for a whole row of key blocks in shared memory (at least B * (L/B)
+ *     * 4 bytes, under about 200 KB); longer layers return RR_ERR_UNSUPPORTED there.  Every
+ *     other supported B/S takes L up to 2^20.
  */
 #ifndef RR_ATTN_H
 #define RR_ATTN_H
@@ -173,8 +173,9 @@ rr_status_t rr_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int 
 
 /*
  * rr_device_errors -- error bits the kernels recorded on the current device instead of
- * trapping: bit 0 producer, bit 1 MMA issuer, bit 2 softmax warps of rr_sparse_prefill gave
- * up a wait after about one second.  *flags (host) receives the bits; reset != 0 clears them.
+ * trapping: bit 0 producer, bit 1 MMA issuer, bit 2 softmax warps of rr_sparse_prefill, bit 3
+ * a warp of rr_estimate's tensor-core kernel gave up a wait after about one second.  *flags
+ * (host) receives the bits; reset != 0 clears them.
  * Synchronous: waits for the device's preceding work.
  */
 rr_status_t rr_device_errors(uint32_t *flags, int reset);

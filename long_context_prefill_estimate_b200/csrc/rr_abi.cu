@@ -24,6 +24,7 @@ rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16
                               int L, int d, int B, const int32_t *row_ptr, const int32_t *col_idx,
                               float scale, uint16_t *O, cudaStream_t st);
 rr_status_t read_device_errors(unsigned *out, bool reset);
+rr_status_t read_estimate_errors(unsigned *out, bool reset);
 
 static thread_local char g_last_error[512] = "";
 
@@ -100,9 +101,10 @@ const char *rr_last_error(void) { return g_last_error; }
 rr_status_t rr_device_errors(uint32_t *flags, int reset) {
     g_last_error[0] = 0;
     if (!flags) return set_error(RR_ERR_INVALID_ARG, "rr_device_errors: flags is NULL");
-    unsigned v = 0;
-    const rr_status_t s = read_device_errors(&v, reset != 0);
-    *flags = v;
+    unsigned v = 0, ve = 0;
+    rr_status_t s = read_device_errors(&v, reset != 0);
+    if (s == RR_OK) s = read_estimate_errors(&ve, reset != 0);
+    *flags = v | ve;
     return s;
 }
 

@@ -14,9 +14,25 @@ rr_status_t check_launch(const char *what);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// TMA descriptor (a CUtensorMap, 128 bytes, 64-byte aligned) of a 2-D row-major bf16 tensor
+// [rows][cols]: boxes of 64 columns x box_rows rows, 128-byte swizzle.  False when the
+// driver entry point is missing or the driver rejects the layout.
+bool make_tmap_bf16(void *tmap, const void *ptr, uint64_t rows, int cols, uint32_t box_rows);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ---------------------------------------------------------------- device helpers
+// Offset inside stride i of the query sampled for query head h (round-robin strategies of
+// Sec. 4.3 Table 6: head h mod S, none S-1, layer l mod S, hybrid (h+l) mod S).
+__device__ __forceinline__ int rr_offset(int h, int S, int mode, int layer) {
+    switch (mode) {
+    case RR_NONE: return S - 1;
+    case RR_LAYER: return layer % S;
+    case RR_HYBRID: return (h + layer) % S;
+    default: return h % S;
+    }
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -87,15 +87,6 @@ struct EstParams {
     float c_log2;  // log2(e) / (S * sqrt(d))
 };
 
-__device__ __forceinline__ int rr_offset(int h, int S, int mode, int layer) {
-    switch (mode) {
-    case RR_NONE: return S - 1;
-    case RR_LAYER: return layer % S;
-    case RR_HYBRID: return (h + layer) % S;
-    default: return h % S;
-    }
-}
-
 template <int D, int MTW, int BPT>
 __global__ void __launch_bounds__(kEstThreads, MTW == 1 ? 2 : 1) estimate_kernel(const EstParams p) {
     constexpr int KS = D / 16;
@@ -331,7 +322,13 @@ size_t estimate_workspace_bytes(int Hkv, int L, int d, int S) {
     return (size_t)Hkv * (L / S) * d * 4;  // bf16 hi + lo per pooled element
 }
 
+bool estimate_tc_eligible(int d, int S, int B);
+rr_status_t launch_estimate_tc(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, int d,
+                               int S, int B, int mode, int layer, int head_base, float *A, void *ws,
+                               cudaStream_t st);
+
 bool estimate_supported(int H, int Hkv, int d, int S, int B, int L) {
+    if (estimate_tc_eligible(d, S, B)) return true;
     EstPlan pl;
     return plan_estimate(H, Hkv, d, S, B, L / B, &pl);
 }
@@ -339,6 +336,10 @@ bool estimate_supported(int H, int Hkv, int d, int S, int B, int L) {
 rr_status_t launch_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, int d,
                             int S, int B, int mode, int layer, int head_base, float *A, void *ws,
                             cudaStream_t st) {
+    // B/S in {4, 8, 16, 32}: the tensor-core (tcgen05) estimator; otherwise (B/S = 64 or
+    // 128, the S = 1 exact mode) the register-fragment kernel below
+    if (estimate_tc_eligible(d, S, B))
+        return launch_estimate_tc(Q, K, H, Hkv, L, d, S, B, mode, layer, head_base, A, ws, st);
     const int Ns = L / S, Nb = L / B;
     EstPlan pl;
     if (!plan_estimate(H, Hkv, d, S, B, Nb, &pl))

@@ -28,8 +28,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include <mutex>
-
 #include "rr_common.cuh"
 #include "rr_sm100.cuh"
 
@@ -40,22 +38,6 @@ namespace {
 __device__ unsigned int g_device_errors;
 
 constexpr unsigned kErrTimeoutProducer = 1u, kErrTimeoutMma = 2u, kErrTimeoutSoftmax = 4u;
-
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for the phase of `parity` to complete, for at most ~1 s.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
-    if (sm100::mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t i = 1;; ++i) {
-        if (sm100::mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 0 && globaltimer() - t0 > 1000000000ull) return false;
-    }
-}
 
 // 2^x on the SFU (approximate, flushes denormals; 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -223,7 +205,7 @@ __global__ void __launch_bounds__(224, 2)
                 }
                 const int s = t % NK;
                 const int y = key_row(t);
-                if (!wait_bar(k_empty(s), ((t / NK) & 1) ^ 1)) {  // S_{t-NK} has completed
+                if (!sm100::mbar_wait(k_empty(s), ((t / NK) & 1) ^ 1)) {  // S_{t-NK} has completed
                     ok = false;
                     break;
                 }
@@ -235,9 +217,9 @@ __global__ void __launch_bounds__(224, 2)
             if (!ok) {
                 atomicOr(&g_device_errors, kErrTimeoutProducer);
                 // let the copies already in flight land before the CTA's memory is released
-                wait_bar(q_full, 0);
+                sm100::mbar_wait(q_full, 0);
                 for (int t = issued > NK ? issued - NK : 0; t < issued; ++t)
-                    wait_bar(k_full(t % NK), (t / NK) & 1);
+                    sm100::mbar_wait(k_full(t % NK), (t / NK) & 1);
             }
         }
     } else if (warp == 1) {
@@ -248,7 +230,7 @@ __global__ void __launch_bounds__(224, 2)
             for (int t = 0; t < nsub; ++t) {
                 const int s = t % NV;
                 const int y = key_row(t);
-                if (!wait_bar(v_empty(s), ((t / NV) & 1) ^ 1)) {  // P_{t-NV} V_{t-NV} has completed
+                if (!sm100::mbar_wait(v_empty(s), ((t / NV) & 1) ^ 1)) {  // P_{t-NV} V_{t-NV} has completed
                     ok = false;
                     break;
                 }
@@ -260,17 +242,17 @@ __global__ void __launch_bounds__(224, 2)
             if (!ok) {
                 atomicOr(&g_device_errors, kErrTimeoutProducer);
                 for (int t = issued > NV ? issued - NV : 0; t < issued; ++t)
-                    wait_bar(v_full(t % NV), (t / NV) & 1);
+                    sm100::mbar_wait(v_full(t % NV), (t / NV) & 1);
             }
         }
     } else if (warp == 2) {
         if (lane == 0) {
             // ---------------------------------------------------------------- MMA issuer
-            bool ok = wait_bar(q_full, 0);
+            bool ok = sm100::mbar_wait(q_full, 0);
             sm100::tc_fence_after();
             auto issue_s = [&](int t) -> bool {
                 const int s = t % NK;
-                if (!wait_bar(k_full(s), (t / NK) & 1)) return false;
+                if (!sm100::mbar_wait(k_full(s), (t / NK) & 1)) return false;
                 sm100::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -287,11 +269,11 @@ __global__ void __launch_bounds__(224, 2)
             if (ok && nsub > 0) ok = issue_s(0);
             for (int t = 0; ok && t < nsub; ++t) {
                 // S_{t+1} goes into the S columns once every softmax thread has loaded S_t
-                if (t + 1 < nsub && !(wait_bar(s_free, t & 1) && issue_s(t + 1))) {
+                if (t + 1 < nsub && !(sm100::mbar_wait(s_free, t & 1) && issue_s(t + 1))) {
                     ok = false;
                     break;
                 }
-                if (!wait_bar(p_full(t), (t >> 1) & 1) || !wait_bar(v_full(t % NV), (t / NV) & 1)) {
+                if (!sm100::mbar_wait(p_full(t), (t >> 1) & 1) || !sm100::mbar_wait(v_full(t % NV), (t / NV) & 1)) {
                     ok = false;
                     break;
                 }
@@ -309,7 +291,7 @@ __global__ void __launch_bounds__(224, 2)
             }
             // fin_bar: every MMA has completed (the epilogue reads O, then the TMEM is released)
             sm100::mma_commit(fin_bar);
-            if (!wait_bar(fin_bar, 0)) ok = false;
+            if (!sm100::mbar_wait(fin_bar, 0)) ok = false;
             if (!ok) atomicOr(&g_device_errors, kErrTimeoutMma);
         }
     } else {
@@ -323,7 +305,7 @@ __global__ void __launch_bounds__(224, 2)
         // A CSR row is ascending with J <= I, so only its last block can be the diagonal one.
         const int tdiag = (nsub > 0 && __ldg(col_idx + e0 + nsub / NSB - 1) == I) ? nsub - NSB : nsub;
         for (int t = 0; t < nsub; ++t) {
-            ok = __all_sync(0xffffffffu, wait_bar(s_full, t & 1));
+            ok = __all_sync(0xffffffffu, sm100::mbar_wait(s_full, t & 1));
             if (!ok) break;
             sm100::tc_fence_after();
             uint32_t sr[kSub];
@@ -385,7 +367,7 @@ __global__ void __launch_bounds__(224, 2)
             f2_unpack(rs2[1], rc, rd);
             l += (ra + rb) + (rc + rd);
             if (t > 0 && __any_sync(0xffffffffu, need)) {
-                ok = __all_sync(0xffffffffu, wait_bar(o_bar, (t - 1) & 1));
+                ok = __all_sync(0xffffffffu, sm100::mbar_wait(o_bar, (t - 1) & 1));
                 if (!ok) break;
                 sm100::tc_fence_after();
 #pragma unroll
@@ -406,7 +388,7 @@ __global__ void __launch_bounds__(224, 2)
         // softmax step ends, only the P*V of two steps earlier is known to be complete, so the
         // barrier may still be two phases short and a parity wait on it would alias.)
         if (ok) {
-            ok = __all_sync(0xffffffffu, wait_bar(fin_bar, 0));
+            ok = __all_sync(0xffffffffu, sm100::mbar_wait(fin_bar, 0));
             sm100::tc_fence_after();
         }
         if (!ok) {
@@ -448,46 +430,14 @@ __global__ void __launch_bounds__(224, 2)
     }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2-D bf16 view [rows][d] of a row-major tensor, boxes of 64 columns x box_rows rows,
-// 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, int d, uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)d, rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int BN>
 rr_status_t launch_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H, int Hkv, int L,
                       const int32_t *row_ptr, const int32_t *col_idx, float scale, uint16_t *O,
                       cudaStream_t st) {
     using C = TcCfg<D, BN>;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, Q, (uint64_t)H * L, D, kBM) || !make_map(&mk, K, (uint64_t)Hkv * L, D, kSub) ||
-        !make_map(&mv, V, (uint64_t)Hkv * L, D, kSub))
+    if (!make_tmap_bf16(&mq, Q, (uint64_t)H * L, D, kBM) || !make_tmap_bf16(&mk, K, (uint64_t)Hkv * L, D, kSub) ||
+        !make_tmap_bf16(&mv, V, (uint64_t)Hkv * L, D, kSub))
         return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cuTensorMapEncodeTiled failed");
     const size_t smem = C::SMEM_LAUNCH;
     auto kern = prefill_tc_kernel<D, BN>;
