@@ -335,6 +335,10 @@ def run_ours(args):
                  + 4 * wl.Hkv * wl.Ns * wl.d * 2    # pooled keys written + read
                  + 4 * wl.H * wl.Nb * wl.Nb)        # block scores written
     sel_bytes = 4 * wl.H * wl.Nb * wl.Nb + 4 * (wl.H * wl.Nb + 1) + 4 * nnz
+    # estimator's algorithmic work: one logit (2*d FLOP) and one exponential per causal
+    # stride pair (i, j <= i) of every query head
+    pairs = wl.H * wl.Ns * (wl.Ns + 1) / 2
+    est_s = stage["estimate_ms"] * 1e-3
     line = {
         "metric": METRIC,
         "value": aggregate_tflops(layers, dense, ms_step),
@@ -348,6 +352,8 @@ def run_ours(args):
         "stages": {**stage,
                    "estimate_gbs": est_bytes / (stage["estimate_ms"] * 1e-3) / 1e9,
                    "select_gbs": sel_bytes / (stage["select_ms"] * 1e-3) / 1e9,
+                   "estimate_tflops": 2 * wl.d * pairs / est_s / 1e12,
+                   "estimate_gexp_per_s": pairs / est_s / 1e9,
                    "prefill_tflops_selected": prefill_tflops},
         "density": nnz / causal_blocks,
         "selected_blocks": nnz, "diag_blocks": n_diag,
@@ -363,6 +369,12 @@ def run_ours(args):
         "gpu_launches": 6 * args.steps,
         "clocks": clocks,
     }
+    # estimator against its two candidate bounds: the bf16 tensor peak (its logits) and the
+    # SFU (16 exp2 per clock per SM x 148 SMs at the measured SM clock)
+    st_ = line["stages"]
+    st_["estimate_frac_tensor"] = st_["estimate_tflops"] / line["roofline"]["peak"]
+    if clocks and clocks.get("sm_mhz"):
+        st_["estimate_frac_sfu"] = st_["estimate_gexp_per_s"] / (16 * 148 * clocks["sm_mhz"] * 1e-3)
     # ---- extra measurements (outside the timed region)
     if rank == 0 and not args.quick:
         line["tau_sweep"] = tau_sweep(wl, step, st, ws, torch)

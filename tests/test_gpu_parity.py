@@ -86,6 +86,7 @@ SMALL = [
     ("gqa7-d64", workloads.get(4, H=14, Hkv=2, L=4096, d=64, S=8, B=64, frame_len=512)),
     ("s32-b128", workloads.get(1, H=8, Hkv=2, L=4096, S=32)),      # B/S = 4: two blocks per tile
     ("s16-b64", workloads.get(0, L=2176, S=16, B=64)),              # B/S = 4 at B = 64
+    ("s4-b128", workloads.get(0, H=4, Hkv=2, L=2048, d=64, S=4, B=128)),  # B/S = 32
 ]
 
 
