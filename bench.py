@@ -479,8 +479,9 @@ def e2e(w, wl, host, h0, layers, rr, torch, dev, args):
     return {"value": aggregate_tflops(layers, dense_causal_flops(w), ms), "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": n,
-            "pipeline": f"{rr.default_chunks(wl.Hkv)} slices of whole KV groups; copy-in, compute "
-                        f"and copy-out on three streams"}
+            "pipeline": f"{len(rr.host_slices(wl.H, wl.Hkv, rr.default_chunks(wl.Hkv)))} slices "
+                        f"(whole KV groups; the first and last query heads alone); copy-in, "
+                        f"compute and copy-out on three streams"}
 
 
 def main(argv=None):

@@ -23,7 +23,7 @@ import torch
 __all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
            "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
            "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors", "default_chunks",
-           "head_shard"]
+           "head_shard", "host_slices"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "librrattn.so")
@@ -274,6 +274,33 @@ def default_chunks(Hkv: int) -> int:
     return max(c for c in range(1, min(Hkv, 8) + 1) if Hkv % c == 0)
 
 
+def host_slices(H: int, Hkv: int, chunks: int, peel: bool = True):
+    """Slices (h0, h1) of the host pipeline: `chunks` ranges of whole KV groups; with `peel`
+    (and more than one query head per group) the layer's first and last query heads become
+    slices of their own, so the first copy-in and the last copy-out are short.  Every slice
+    is whole KV groups or heads of a single group."""
+    G = H // Hkv
+    gc = Hkv // chunks
+    units = [(c * gc * G, (c + 1) * gc * G) for c in range(chunks)]
+    if not peel or G == 1:
+        return units
+    out = []
+    for i, (h0, h1) in enumerate(units):
+        parts = [(h0, h1)]
+        if i == 0:  # head h0 | the rest of its group | the remaining whole groups
+            parts = [(h0, h0 + 1), (h0 + 1, h0 + G)] + ([(h0 + G, h1)] if h1 > h0 + G else [])
+        if i == len(units) - 1:  # ... | the last group but its last head | the last head
+            a, b = parts.pop()
+            if b - a > G:
+                parts.append((a, b - G))
+                a = b - G
+            if b - 1 > a:
+                parts.append((a, b - 1))
+            parts.append((b - 1, b))
+        out += parts
+    return out
+
+
 def _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, scale, out, chunks,
                             head_base=0):
     for n, t in (("Q", Q), ("K", K), ("V", V)):
@@ -290,38 +317,45 @@ def _prefill_host_pipelined(Q, K, V, S, B, tau, protect_last, strategy, layer, s
     if dst.shape != Q.shape or dst.dtype != Q.dtype or dst.is_cuda or not dst.is_contiguous():
         raise RRAttnError("prefill", 1, "out must be a contiguous bf16 host tensor shaped like Q")
     dev = torch.device("cuda", torch.cuda.current_device())
-    gc, hc = Hkv // n, H // n
+    G, Nb = H // Hkv, (L // B if B > 0 else 0)
+    # heads of one group may form a slice only where the estimator's per-row arithmetic does
+    # not depend on how many heads share a CTA (B/S <= 32); there the bytes match one pass
+    slices = host_slices(H, Hkv, n, peel=B > 0 and S > 0 and (B // S) in (4, 8, 16, 32))
+    spans = [(h0, h1, h0 // G, (h1 - 1) // G + 1) for h0, h1 in slices]
+    mh = max(h1 - h0 for h0, h1, _, _ in spans)
+    mg = max(g1 - g0 for _, _, g0, g1 in spans)
     compute = torch.cuda.current_stream(dev)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     Qd, Kd, Vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (Q, K, V))
     Od = torch.empty(Q.shape, dtype=Q.dtype, device=dev)
-    ws = Workspace(hc, gc, L, d, S, B, device=dev)
+    ws = Workspace(mh, mg, L, d, S, B, device=dev)
     # the fresh buffers may reuse memory last used on the compute stream
     s_in.wait_stream(compute)
     s_out.wait_stream(compute)
-    loaded = []
+    loaded, kv_done = [], 0
     with torch.cuda.stream(s_in):
-        for c in range(n):
-            hs, gs = slice(c * hc, (c + 1) * hc), slice(c * gc, (c + 1) * gc)
-            Qd[hs].copy_(Q[hs], non_blocking=True)
-            Kd[gs].copy_(K[gs], non_blocking=True)
-            Vd[gs].copy_(V[gs], non_blocking=True)
+        for h0, h1, g0, g1 in spans:
+            Qd[h0:h1].copy_(Q[h0:h1], non_blocking=True)
+            if g1 > kv_done:  # each group's K/V travels with the first slice that needs it
+                Kd[kv_done:g1].copy_(K[kv_done:g1], non_blocking=True)
+                Vd[kv_done:g1].copy_(V[kv_done:g1], non_blocking=True)
+                kv_done = g1
             ev = torch.cuda.Event()
             ev.record(s_in)
             loaded.append(ev)
-    for c in range(n):
-        hs, gs = slice(c * hc, (c + 1) * hc), slice(c * gc, (c + 1) * gc)
-        compute.wait_event(loaded[c])
-        estimate(Qd[hs], Kd[gs], S, B, strategy=strategy, layer=layer, out=ws.block_scores,
-                 workspace=ws.est, head_base=head_base + c * hc)
-        select(ws.block_scores, tau, protect_last, row_ptr=ws.row_ptr, col_idx=ws.col_idx,
-               nnz=ws.nnz, workspace=ws.sel)
-        sparse_prefill(Qd[hs], Kd[gs], Vd[gs], ws.row_ptr, ws.col_idx, B, scale=scale, out=Od[hs])
+    for (h0, h1, g0, g1), ev in zip(spans, loaded):
+        nh = h1 - h0
+        A, rp = ws.block_scores[:nh], ws.row_ptr[:nh * Nb + 1]
+        compute.wait_event(ev)
+        estimate(Qd[h0:h1], Kd[g0:g1], S, B, strategy=strategy, layer=layer, out=A,
+                 workspace=ws.est, head_base=head_base + h0)
+        select(A, tau, protect_last, row_ptr=rp, col_idx=ws.col_idx, nnz=ws.nnz, workspace=ws.sel)
+        sparse_prefill(Qd[h0:h1], Kd[g0:g1], Vd[g0:g1], rp, ws.col_idx, B, scale=scale, out=Od[h0:h1])
         done = torch.cuda.Event()
         done.record(compute)
         s_out.wait_event(done)
         with torch.cuda.stream(s_out):
-            dst[hs].copy_(Od[hs], non_blocking=True)
+            dst[h0:h1].copy_(Od[h0:h1], non_blocking=True)
     s_out.synchronize()
     # every copy and kernel above has completed; later work on the compute stream may
     # reuse the buffers

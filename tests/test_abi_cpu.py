@@ -104,6 +104,25 @@ def test_host_path_argument_checks(L):
         rr.prefill(Q.float(), K, K, 8, 64, 0.9)
 
 
+def test_host_pipeline_slices():
+    # contiguous, covering, each slice whole KV groups or heads of one group; the first and
+    # last query heads stand alone when a group has several heads
+    for H, Hkv in [(32, 8), (28, 4), (4, 1), (2, 2), (16, 4), (8, 8), (14, 2)]:
+        G = H // Hkv
+        for chunks in [c for c in range(1, Hkv + 1) if Hkv % c == 0]:
+            for peel in (True, False):
+                sl = rr.host_slices(H, Hkv, chunks, peel)
+                assert sl[0][0] == 0 and sl[-1][1] == H
+                assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
+                for h0, h1 in sl:
+                    assert h1 > h0
+                    assert (h1 - 1) // G == h0 // G or (h0 % G == 0 and h1 % G == 0)
+                if peel and G > 1:
+                    assert sl[0] == (0, 1) and sl[-1] == (H - 1, H)
+                if not peel:
+                    assert len(sl) == chunks
+
+
 def test_select_rejections(L):
     P = FAKE
     ok_cap = 2 * 4 * 5 // 2
