@@ -180,6 +180,16 @@ rr_status_t rr_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int 
  */
 rr_status_t rr_device_errors(uint32_t *flags, int reset);
 
+/*
+ * rr_selftest_wait -- exercises the bounded wait the kernels use in place of an unbounded
+ * spin (no counterpart in the paper).  A one-thread kernel waits on an mbarrier phase that
+ * nothing completes; after timeout_us (1 .. 2,000,000) it must give up; it then completes the
+ * phase itself and waits again, which must succeed.  result (host, 3 elements): [0] = 1 if
+ * the first wait gave up, [1] = 1 if the second saw the phase, [2] = microseconds the first
+ * wait took.  Synchronous on the legacy default stream; touches no other library state.
+ */
+rr_status_t rr_selftest_wait(uint32_t timeout_us, uint32_t *result);
+
 /* Static text for a status code. */
 const char *rr_status_string(rr_status_t s);
 

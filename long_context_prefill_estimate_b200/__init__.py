@@ -23,7 +23,7 @@ import torch
 __all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
            "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
            "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors", "default_chunks",
-           "head_shard", "host_slices"]
+           "head_shard", "host_slices", "selftest_wait"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "librrattn.so")
@@ -34,7 +34,8 @@ EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_heads",
                     "rr_estimate_workspace_bytes",
                     "rr_select", "rr_select_workspace_bytes", "rr_select_noalloc",
                     "rr_sparse_prefill",
-                    "rr_validate_csr", "rr_device_errors", "rr_status_string", "rr_last_error",
+                    "rr_validate_csr", "rr_device_errors", "rr_selftest_wait", "rr_status_string",
+                    "rr_last_error",
                     "rr_version")
 
 
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.rr_validate_csr.restype = I
     L.rr_device_errors.argtypes = [P, I]
     L.rr_device_errors.restype = I
+    L.rr_selftest_wait.argtypes = [ctypes.c_uint32, P]
+    L.rr_selftest_wait.restype = I
     L.rr_status_string.argtypes = [I]
     L.rr_status_string.restype = ctypes.c_char_p
     L.rr_last_error.argtypes = []
@@ -370,6 +373,13 @@ def validate_csr(row_ptr: torch.Tensor, col_idx: torch.Tensor, H: int, Nb: int) 
     _check("rr_validate_csr", lib().rr_validate_csr(
         _ptr(row_ptr), _ptr(col_idx), H, Nb, col_idx.numel(), _ptr(bad), _stream(row_ptr.device)))
     return int(bad.item())
+
+
+def selftest_wait(timeout_us: int = 20000) -> Tuple[bool, bool, int]:
+    """Runs the bounded-wait self-test: (gave_up, saw_completed_phase, microseconds)."""
+    r = (ctypes.c_uint32 * 3)()
+    _check("rr_selftest_wait", lib().rr_selftest_wait(int(timeout_us), r))
+    return bool(r[0]), bool(r[1]), int(r[2])
 
 
 def device_errors(reset: bool = True) -> int:

@@ -25,6 +25,7 @@ rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16
                               float scale, uint16_t *O, cudaStream_t st);
 rr_status_t read_device_errors(unsigned *out, bool reset);
 rr_status_t read_estimate_errors(unsigned *out, bool reset);
+rr_status_t selftest_wait(uint32_t timeout_us, uint32_t *result);
 
 static thread_local char g_last_error[512] = "";
 
@@ -106,6 +107,15 @@ rr_status_t rr_device_errors(uint32_t *flags, int reset) {
     if (s == RR_OK) s = read_estimate_errors(&ve, reset != 0);
     *flags = v | ve;
     return s;
+}
+
+rr_status_t rr_selftest_wait(uint32_t timeout_us, uint32_t *result) {
+    g_last_error[0] = 0;
+    if (!result) return set_error(RR_ERR_INVALID_ARG, "rr_selftest_wait: result is NULL");
+    if (timeout_us == 0 || timeout_us > 2000000u)
+        return set_error(RR_ERR_INVALID_ARG, "rr_selftest_wait: timeout_us=%u outside (0, 2e6]",
+                         timeout_us);
+    return selftest_wait(timeout_us, result);
 }
 
 size_t rr_estimate_workspace_bytes(int H, int Hkv, int L, int d, int S, int B) {

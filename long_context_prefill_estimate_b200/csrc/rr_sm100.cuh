@@ -39,14 +39,16 @@ __device__ __forceinline__ uint64_t globaltimer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for the phase of `parity` to complete, for at most about one second of %globaltimer;
-// false when it gave up (the caller records an error and drains instead of hanging).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of `parity` to complete, for at most limit_ns of %globaltimer (about
+// one second by default); false when it gave up (the caller records an error and drains
+// instead of hanging).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint64_t limit_ns = 1000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 0 && globaltimer() - t0 > 1000000000ull) return false;
+        if ((i & 1023u) == 0 && globaltimer() - t0 > limit_ns) return false;
     }
 }
 

@@ -104,6 +104,14 @@ def test_host_path_argument_checks(L):
         rr.prefill(Q.float(), K, K, 8, 64, 0.9)
 
 
+def test_selftest_wait_rejections(L):
+    buf = (ctypes.c_uint32 * 3)()
+    assert L.rr_selftest_wait(0, buf) == INVALID
+    assert L.rr_selftest_wait(3000000, buf) == INVALID
+    assert L.rr_selftest_wait(1000, None) == INVALID
+    assert b"timeout_us" in L.rr_last_error() or b"result" in L.rr_last_error()
+
+
 def test_host_pipeline_slices():
     # contiguous, covering, each slice whole KV groups or heads of one group; the first and
     # last query heads stand alone when a group has several heads

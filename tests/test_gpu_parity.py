@@ -202,6 +202,19 @@ def test_extreme_softmax_scales(scale, cuda_device):
     _check_output(O.float().cpu()[idx[:, 0], idx[:, 1]].numpy(), O_ref)
 
 
+def test_bounded_wait_gives_up_and_device_stays_usable(cuda_device):
+    # the wait every kernel uses instead of an unbounded spin: on a phase nothing completes
+    # it gives up after its limit (here 20 ms), and a completed phase is still seen
+    gave_up, saw, us = rr.selftest_wait(20000)
+    assert gave_up and saw
+    assert 20000 <= us < 1000000
+    w = workloads.get(0)
+    t = _to(workloads.generate(w), cuda_device)
+    A = rr.estimate(t["Q"], t["K"], w.S, w.B)
+    torch.cuda.synchronize()
+    assert torch.isfinite(A).all() and rr.device_errors() == 0
+
+
 def test_no_device_errors_recorded(cuda_device):
     assert rr.device_errors(reset=False) == 0
 
