@@ -215,6 +215,22 @@ def test_bounded_wait_gives_up_and_device_stays_usable(cuda_device):
     assert torch.isfinite(A).all() and rr.device_errors() == 0
 
 
+@pytest.mark.parametrize("gain", [8.0, 0.05])
+def test_estimate_sharp_and_flat_attention(gain, cuda_device):
+    # logits scaled up (one stride dominates each row; the lazy max rescale fires) or down
+    # (nearly uniform rows): block scores still match the oracle and rows sum to 1
+    w = workloads.get(1, H=8, Hkv=2, L=4096)
+    t = workloads.generate(w)
+    for k in ("Q", "K"):
+        t[k] = (t[k].float() * (gain ** 0.5)).to(torch.bfloat16)
+    d = _to(t, cuda_device)
+    A = rr.estimate(d["Q"], d["K"], w.S, w.B).cpu().numpy().astype(np.float64)
+    A_or = oracle.estimate(t["Q"], t["K"], w.S, w.B)
+    assert np.abs(A - A_or).max() <= SCORE_TOL
+    assert np.allclose(A.sum(-1), 1.0, atol=1e-5)
+    assert rr.device_errors() == 0
+
+
 def test_no_device_errors_recorded(cuda_device):
     assert rr.device_errors(reset=False) == 0
 
