@@ -69,13 +69,6 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// 2^x on the SFU (relative error about 2^-22; 2^-inf = 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 struct EstParams {
     const uint16_t *Q;
     const uint4 *frag;

@@ -34,12 +34,6 @@ constexpr unsigned kErrTimeoutEstimate = 8u;
 constexpr int kRows = 128;   // sampled rows per CTA (tensor-core M)
 constexpr int kTileN = 128;  // strides per key tile (tensor-core N)
 
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 template <int D>
 __global__ void __launch_bounds__(256) pool_keys_rows_kernel(const uint16_t *__restrict__ K, int L, int S,
                                                              int Ns, int Hkv, uint16_t *__restrict__ hi,

@@ -39,13 +39,6 @@ __device__ unsigned int g_device_errors;
 
 constexpr unsigned kErrTimeoutProducer = 1u, kErrTimeoutMma = 2u, kErrTimeoutSoftmax = 4u;
 
-// 2^x on the SFU (approximate, flushes denormals; 2^-inf = 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // max(a, b, c) in one instruction (sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float y;
