@@ -231,6 +231,31 @@ def test_estimate_sharp_and_flat_attention(gain, cuda_device):
     assert rr.device_errors() == 0
 
 
+def test_maximum_sequence_length(cuda_device):
+    # L = 2^20, the longest layer the ABI accepts: 8192 key blocks per row (the long-row
+    # selection path), properties of the scores, a valid CSR, and sampled output rows against
+    # the oracle under the GPU's CSR
+    w = workloads.get(1, H=2, Hkv=1, L=1 << 20)
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    A = rr.estimate(d["Q"], d["K"], w.S, w.B)
+    rp, ci, nnz = rr.select(A, w.tau, True)
+    O = rr.sparse_prefill(d["Q"], d["K"], d["V"], rp, ci, w.B)
+    torch.cuda.synchronize()
+    assert rr.device_errors() == 0
+    Nb = w.Nb
+    assert torch.allclose(A.sum(-1), torch.ones(w.H, Nb, device=A.device), atol=1e-4)
+    assert torch.count_nonzero(torch.triu(A, diagonal=1)) == 0
+    n = int(nnz.item())
+    assert rr.validate_csr(rp, ci[:n].contiguous(), w.H, Nb) == 0
+    rp_h, ci_h = rp.cpu().numpy(), ci[:n].cpu().numpy()
+    rng = np.random.default_rng(7)
+    rows = [(h, int(q)) for h in range(w.H) for q in rng.integers(0, w.L, 3)] + [(1, w.L - 1)]
+    O_ref = oracle.prefill_rows(t["Q"], t["K"], t["V"], w.B, rp_h, ci_h, rows)
+    idx = torch.as_tensor(rows)
+    _check_output(O.float().cpu()[idx[:, 0], idx[:, 1]].numpy(), O_ref)
+
+
 def test_no_device_errors_recorded(cuda_device):
     assert rr.device_errors(reset=False) == 0
 
