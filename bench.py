@@ -366,7 +366,9 @@ def run_ours(args):
                      "flops_per_launch": sel_flops,
                      "traffic": prefill_traffic_per_launch(wl),
                      "traffic_unit": "bytes/launch (ncu dram read+write at L=32768, scaled by L)"},
-        "gpu_launches": 6 * args.steps,
+        # per step: key pooling, estimate, select (warp-per-row kernel, plus the sorting kernel
+        # when rows exceed 1024 blocks), count scan, CSR emit, prefill
+        "gpu_launches": (6 + (1 if wl.Nb > 1024 else 0)) * args.steps,
         "clocks": clocks,
     }
     # estimator against its two candidate bounds: the bf16 tensor peak (its logits) and the
