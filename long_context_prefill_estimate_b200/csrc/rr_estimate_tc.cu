@@ -9,8 +9,10 @@
 //                          queries Q[h][i*S + off(h)] of those heads and blocks (QB * hc * r
 //                          of them, r = B/S), staged once into shared memory in the tensor
 //                          core's 128-byte-swizzled layout.  Pooled keys arrive by TMA in
-//                          tiles of 128 strides; S = Qhat (Kbar_hi + Kbar_lo)^T (fp32-grade
-//                          logits) goes to one of two TMEM buffers.  Two passes over the
+//                          tiles of 64 strides; S = Qhat (Kbar_hi + Kbar_lo)^T (fp32-grade
+//                          logits) goes to one of two TMEM buffers.  96 KB of shared memory
+//                          and 128 TMEM columns per CTA: two CTAs share an SM, so the
+//                          softmax of one overlaps the MMAs and loads of the other.  Two passes over the
 //                          tiles: the first finds each row's max and sum of exp2 over the
 //                          causal strides j <= i; the second recomputes S, normalises exactly,
 //                          sums each key block's r strides and reduces over the r rows of each
@@ -32,7 +34,7 @@ __device__ unsigned int g_est_errors;
 constexpr unsigned kErrTimeoutEstimate = 8u;
 
 constexpr int kRows = 128;   // sampled rows per CTA (tensor-core M)
-constexpr int kTileN = 128;  // strides per key tile (tensor-core N)
+constexpr int kTileN = 64;   // strides per key tile (tensor-core N)
 
 template <int D>
 __global__ void __launch_bounds__(256) pool_keys_rows_kernel(const uint16_t *__restrict__ K, int L, int S,
@@ -86,17 +88,17 @@ struct EstTcCfg {
     static constexpr int DC = D / 64;
     static constexpr uint32_t Q_BYTES = kRows * D * 2;
     static constexpr uint32_t T_BYTES = kTileN * D * 2;  // one hi or lo key tile
-    static constexpr int NS = D == 128 ? 3 : 4;          // stages of (hi, lo) tiles
+    static constexpr int NS = D == 128 ? 2 : 4;          // stages of (hi, lo) tiles
     static constexpr uint32_t BAR_OFF = Q_BYTES + NS * 2 * T_BYTES;
     // k_full[NS], k_empty[NS], s_full[2], s_free[2], fin
     static constexpr uint32_t NBAR = 2 * NS + 5;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
     static constexpr uint32_t IDESC = sm100::idesc_bf16(kRows, kTileN, false);
-    static_assert(SMEM + 1024 <= 227u * 1024u, "shared memory budget");
+    static_assert(SMEM + 1024 <= 113u * 1024u, "two CTAs per SM");
 };
 
 template <int D, int R>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
     estimate_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__ CUtensorMap tmLo,
                        const EstTcParams p) {
     using C = EstTcCfg<D>;
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(256, 1)
         sm100::fence_mbar_init();
     }
     if (warp == 0) {
-        sm100::tmem_alloc(smem_u32(tmem_slot), 256);
+        sm100::tmem_alloc(smem_u32(tmem_slot), 2 * kTileN);
         sm100::tmem_relinquish();
     }
     // Stage the sampled rows: row rho = qb*RB + hh*r + ii samples stride i = (I0+qb)*r + ii of
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(256, 1)
     if (warp == 0) {
         __syncwarp();  // lane 0 ran the producer; dealloc is warp-collective
         sm100::tc_fence_after();
-        sm100::tmem_dealloc(tmem, 256);
+        sm100::tmem_dealloc(tmem, 2 * kTileN);
     }
 }
 
