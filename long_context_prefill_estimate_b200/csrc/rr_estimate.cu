@@ -2,7 +2,10 @@
 // via Per-Head Round-Robin Shifts for Long-Context Inference", Sec. 3.1 heading, Sec. 3.2,
 // Sec. 3.3 heading).
 //
-// Two kernels:
+// launch_estimate sends B/S in {4, 8, 16, 32} to the tensor-core (tcgen05) estimator of
+// rr_estimate_tc.cu.  This file holds the launch planning and, for B/S = 64 or 128 (S = 1,
+// the exact mode), a register-fragment estimator whose rows of a query block span several
+// warps:
 //   pool_keys_kernel  Kbar_j = sum of the S keys of stride j (fp32), split into bf16 hi + lo
 //                     and stored directly in the register order of the m16n8k16 B operand.
 //                     HBM bound: reads K once, writes Hkv*Ns*d*4 bytes.
