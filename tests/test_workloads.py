@@ -41,3 +41,20 @@ def test_video_frames_correlated():
     K = workloads.generate(w)["K"].float()
     same = torch.nn.functional.cosine_similarity(K[0, 10], K[0, 900], dim=0)
     assert same > 0.6
+
+
+def test_bench_flop_accounting():
+    # with every causal block selected, the selected-block FLOPs (4*B*B*d per off-diagonal
+    # block, 4*d*B*(B+1)/2 per diagonal block) equal the dense causal FLOPs 4*d*H*L*(L+1)/2
+    import os
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import oracle
+
+    for w in (workloads.get(0), workloads.get(1, H=3, Hkv=1, L=1024), workloads.get(4, L=2048)):
+        rp, ci = oracle.full_csr(w.H, w.Nb)
+        flops, n_diag, n_off = bench.selected_flops(rp, ci, w.H, w.Nb, w.B, w.d)
+        assert n_diag == w.H * w.Nb and n_off == w.H * w.Nb * (w.Nb - 1) // 2
+        assert flops == bench.dense_causal_flops(w)
