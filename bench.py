@@ -8,8 +8,9 @@ L = 131072, 32/8 heads, d = 128, S = 16, B = 128, tau = 0.9) on seeded synthetic
 Prints one JSON line.  ``value`` is effective TFLOP/s: dense-causal attention FLOPs
 4*d*H*L(L+1)/2 per layer, times the layers all ranks processed, divided by the max-over-ranks
 device time.  Under torchrun each rank runs its own layer (independent problems, weak
-scaling, no data-path collective).  ``--impl reference`` times the CPU oracle on a bounded
-sample of the same workload (rank 0 only).
+scaling, no data-path collective); with ``--shard heads`` the ranks split one layer by whole
+KV groups instead (strong scaling, still no data-path collective).  ``--impl reference``
+times the CPU oracle on a bounded sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
