@@ -23,10 +23,6 @@
  *   - L = 0 is accepted by every call as an empty problem: nothing is launched.
  *   - Supported: d in {64, 128}; B in {64, 128}; 1 <= S <= B with B % S == 0 and B/S = 4
  *     or a multiple of 8; (L/S) % 8 == 0; L % B == 0; H % Hkv == 0; L <= 2^20; H <= 256.
- *     For B/S = 64 or 128 (S = 1, the exact mode) rr_estimate keeps, per CTA, the block sums
- *     of its sampled rows for a whole row of key blocks in shared memory (at least B * (L/B)
- *     * 4 bytes, under about 200 KB); longer layers return RR_ERR_UNSUPPORTED there.  Every
- *     other supported B/S takes L up to 2^20.
  */
 #ifndef RR_ATTN_H
 #define RR_ATTN_H

@@ -152,8 +152,7 @@ rr_status_t rr_estimate_heads(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int
                          workspace ? workspace_bytes : (size_t)0);
     RR_TRY(check_ptr(fn, "workspace", workspace));
     if (!estimate_supported(H, Hkv, d, S, B, L))
-        return set_error(RR_ERR_UNSUPPORTED, "%s: no launch plan fits (H=%d Hkv=%d L=%d S=%d B=%d)",
-                         fn, H, Hkv, L, S, B);
+        return set_error(RR_ERR_UNSUPPORTED, "%s: no kernel for d=%d B/S=%d", fn, d, B / S);
     return launch_estimate(Q, K, H, Hkv, L, d, S, B, (int)strategy, layer, head_base, block_scores,
                            workspace, static_cast<cudaStream_t>(stream));
 }

@@ -75,10 +75,6 @@ def test_estimate_rejections(L):
     assert _est(L, wsb=16) == WORKSPACE
     assert b"workspace" in L.rr_last_error()
     assert _est(L, Len=0, q=0, k=0, out=0, ws=0) == 0   # empty problem: accepted, no launch
-    # in the S = 1 (exact) mode the estimator keeps a row of block sums per CTA in shared
-    # memory: 64 rows x 1024 key blocks x 4 bytes is past its budget
-    assert _est(L, H=2, Hkv=2, Len=65536, d=64, S=1, B=64) == UNSUPPORTED
-    assert b"no launch plan" in L.rr_last_error()
 
 
 def test_estimate_heads_rejections(L):
