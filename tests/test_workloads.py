@@ -58,3 +58,32 @@ def test_bench_flop_accounting():
         flops, n_diag, n_off = bench.selected_flops(rp, ci, w.H, w.Nb, w.B, w.d)
         assert n_diag == w.H * w.Nb and n_off == w.H * w.Nb * (w.Nb - 1) // 2
         assert flops == bench.dense_causal_flops(w)
+
+
+def test_bench_traffic_comes_from_the_matching_capture(tmp_path, monkeypatch):
+    # the roofline's DRAM traffic is the committed ncu capture at 32K scaled by L, for the
+    # captured shape only, and only while the kernel source matches the capture's hash
+    import os
+    import shutil
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+
+    w32, w128 = workloads.get(1), workloads.get(2)
+    t32 = bench.prefill_traffic_per_launch(w32)
+    if t32 is None:  # the capture predates the current kernel source: nothing to check
+        return
+    assert bench.prefill_traffic_per_launch(w128) == 4 * t32
+    assert bench.prefill_traffic_per_launch(workloads.get(0)) is None      # other shape
+    # a changed kernel source invalidates the capture
+    fake = tmp_path / "repo"
+    (fake / "profiles").mkdir(parents=True)
+    (fake / "long_context_prefill_estimate_b200" / "csrc").mkdir(parents=True)
+    shutil.copy(os.path.join(root, "profiles", "prefill_tc_llama3-8b-layer-L32k.md"), fake / "profiles")
+    src = os.path.join(root, "long_context_prefill_estimate_b200", "csrc", "rr_prefill_tc.cu")
+    (fake / "long_context_prefill_estimate_b200" / "csrc" / "rr_prefill_tc.cu").write_text(
+        open(src).read() + "\n// edited\n")
+    monkeypatch.setattr(bench, "ROOT", str(fake))
+    assert bench.prefill_traffic_per_launch(w32) is None
