@@ -27,6 +27,10 @@ MUTANTS = {
     "GQA group by modulo": ("const int g = h / G;\n            const long r", "const int g = h % Hkv;\n            const long r"),
     "softmax without max shift uses wrong sign": ("p[j] = exp(p[j] - m);", "p[j] = exp(m - p[j]);"),
     "transposed block accumulation": ("Arow[j / r] += w * p[j];", "Arow[(j / r) % (I + 1)] += w * p[i - j];"),
+    "diag cum_before reports cum_at": ("diag[1] = cum_before;", "diag[1] = cum;"),
+    "diag threshold without tau": ("diag[3] = thr;", "diag[3] = T;"),
+    "diag gap one past the cut": ("(kstar < n) ? buf[kstar - 1].a - buf[kstar].a",
+                                  "(kstar + 1 < n) ? buf[kstar].a - buf[kstar + 1].a"),
 }
 
 

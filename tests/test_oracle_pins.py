@@ -200,6 +200,59 @@ def test_select_hand_worked(scores, tau, expected):
     assert ci[rp[n - 1]:rp[n]].tolist() == expected
 
 
+def _golden_select_diag():
+    out = []
+    with open(os.path.join(GOLDEN, "select_diag_worked_example.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            sc, tau, exp = line.split(";")
+            out.append(([float(x) for x in sc.split()], float(tau), [float(x) for x in exp.split()]))
+    return out
+
+
+@pytest.mark.parametrize("scores,tau,expected", _golden_select_diag())
+def test_select_diag_hand_worked(scores, tau, expected):
+    # the per-row diagnostics the GPU parity tests classify mismatching rows with: k*, the
+    # cumulative sums on both sides of the cut, tau*T and the score gap across the cut
+    n = len(scores)
+    A = np.zeros((1, n, n))
+    A[0, n - 1, :] = scores
+    rp, ci, dg = oracle.select(A, tau, protect_last=False, diag=True)
+    got = dg[n - 1]
+    assert int(got[0]) == int(expected[0]) == rp[n] - rp[n - 1]
+    np.testing.assert_allclose(got[1:4], expected[1:4], rtol=0, atol=1e-12)
+    if math.isinf(expected[4]):
+        assert math.isinf(got[4]) and got[4] > 0
+    else:
+        assert got[4] == pytest.approx(expected[4], abs=1e-12)
+
+
+def test_select_diag_bruteforce():
+    # the diagnostics against their definitions, recomputed from a brute-force sort
+    rng = np.random.default_rng(3)
+    for trial in range(40):
+        n = int(rng.integers(1, 40))
+        a = rng.gamma(0.3, size=n)
+        if trial % 4 == 0:
+            a = np.round(a * 4) / 4
+        tau = float(rng.choice([0.5, 0.8, 0.9, 0.95]))
+        A = np.zeros((1, n, n))
+        A[0, n - 1] = a
+        _, _, dg = oracle.select(A, tau, protect_last=False, diag=True)
+        order = sorted(range(n), key=lambda j: (-a[j], j))
+        s = a[order]
+        cum = np.cumsum(s)   # sequential sums in the sorted order
+        T = cum[-1]
+        k = int(np.argmax(cum >= tau * T)) + 1
+        assert int(dg[n - 1, 0]) == k
+        assert dg[n - 1, 1] == pytest.approx(cum[k - 2] if k > 1 else 0.0, abs=1e-12)
+        assert dg[n - 1, 2] == pytest.approx(cum[k - 1], abs=1e-12)
+        assert dg[n - 1, 3] == pytest.approx(tau * T, abs=1e-12)
+        gap = s[k - 1] - s[k] if k < n else math.inf
+        assert dg[n - 1, 4] == pytest.approx(gap, abs=1e-12)
+
+
 def test_select_bruteforce_minimal():
     rng = np.random.default_rng(0)
     for trial in range(60):
