@@ -2,11 +2,19 @@
 
 Tolerances:
   block scores  |GPU - oracle| <= 1e-5 (fp32 kernel vs float64 oracle)
-  masks         bit-exact on every non-boundary row.  A row is a boundary row when the
-                oracle's cumulative sum just before or at the cut is within 1e-4 of tau*T,
-                or the scores on either side of the cut differ by less than 1e-5 (then a
-                score error may swap them).  Boundary rows are counted and reported.
-                Selection from identical fp32 scores must match on every row.
+  masks         Selection from identical scores must match the oracle on every row.  End
+                to end (each side selecting from its own scores) every row must match,
+                except rows of these kinds, which are counted and reported:
+                  boundary   the oracle's cumulative sum just before or at the cut is within
+                             1e-4 of tau*T (the boundary rule of the target);
+                  near tie   the same number of blocks, and every block the two sides
+                             disagree on has an oracle score within 2*delta of the oracle's
+                             cut score, delta = the row's largest |GPU - oracle| score error
+                             (a score error of delta can swap only such blocks);
+                  sum within error  the counts differ and the cumulative sum at or before
+                             the cut is within 2*n*delta of tau*T (n blocks in the row).
+                Any other mismatch fails.  With RR_PARITY_RECORD=<dir> the full-size test
+                writes the per-layer counts to <dir>/mask_parity_<layer>.json.
   output O      max-abs <= 2e-2 and rel-L2 <= 1e-2 (bf16 kernel vs float64 oracle), with
                 both sides using the GPU's CSR.
 """
@@ -24,7 +32,6 @@ pytestmark = pytest.mark.gpu
 
 SCORE_TOL = 1e-5
 CUM_TOL = 1e-4
-GAP_TOL = 1e-5
 
 
 def _to(t, dev):
@@ -38,8 +45,9 @@ def _csr_rows(rp, ci):
 
 
 def _boundary_rows(diag):
+    """Rows whose cumulative sum just before or at the cut is within 1e-4 of tau*T."""
     kstar, cb, ca, thr, gap = diag.T
-    return (np.abs(cb - thr) < CUM_TOL) | (np.abs(ca - thr) < CUM_TOL) | (gap < GAP_TOL)
+    return (np.abs(cb - thr) < CUM_TOL) | (np.abs(ca - thr) < CUM_TOL)
 
 
 def _gpu_pipeline(w, t, dev, tau=None, protect_last=True, strategy="head", layer=0):
@@ -56,14 +64,45 @@ def _gpu_pipeline(w, t, dev, tau=None, protect_last=True, strategy="head", layer
     return A.cpu().numpy(), rp_h, ci[:n].cpu().numpy(), O
 
 
-def _check_masks(gpu_rows, rp_o, ci_o, diag):
+def _classify_masks(gpu_rows, rp_o, ci_o, diag, A_or, A_gpu):
+    """Compare the GPU's rows with the oracle's.  Row r of both lists is query block
+    I = r % Nb of a head (the lists start at a head boundary); A_or and A_gpu are the two
+    sides' scores of the same rows, [rows][Nb].  Returns the counts of the module docstring
+    and the rows no case explains."""
     orc_rows = _csr_rows(rp_o, ci_o)
+    Nb = A_or.shape[-1]
     bnd = _boundary_rows(diag)
-    mism = [r for r in range(len(orc_rows)) if gpu_rows[r] != orc_rows[r]]
-    bad = [r for r in mism if not bnd[r]]
-    assert not bad, f"{len(bad)} non-boundary rows differ, e.g. row {bad[0]}: " \
-                    f"gpu {gpu_rows[bad[0]]} oracle {orc_rows[bad[0]]}"
-    return int(bnd.sum()), len(mism)
+    out = {"rows": len(orc_rows), "boundary_rows": int(bnd.sum()), "mismatch_rows": 0,
+           "mismatch_boundary": 0, "near_tie_swaps": 0, "sum_within_error": 0}
+    unexplained = []
+    for r, (g, o) in enumerate(zip(gpu_rows, orc_rows)):
+        if g == o:
+            continue
+        out["mismatch_rows"] += 1
+        if bnd[r]:
+            out["mismatch_boundary"] += 1
+            continue
+        n = r % Nb + 1                      # causal blocks of the row
+        a_or = np.asarray(A_or[r], np.float64)
+        delta = float(np.abs(np.asarray(A_gpu[r], np.float64)[:n] - a_or[:n]).max())
+        cut = float(a_or[o].min())          # the oracle's k*-th score
+        diff = sorted(set(g) ^ set(o))
+        if len(g) == len(o) and all(abs(a_or[J] - cut) <= 2 * delta for J in diff):
+            out["near_tie_swaps"] += 1
+            continue
+        _, cb, ca, thr, _ = diag[r]
+        if len(g) != len(o) and min(abs(cb - thr), abs(ca - thr)) <= 2 * n * delta:
+            out["sum_within_error"] += 1
+            continue
+        unexplained.append((r, g, o))
+    return out, unexplained
+
+
+def _check_masks(gpu_rows, rp_o, ci_o, diag, A_or, A_gpu):
+    counts, bad = _classify_masks(gpu_rows, rp_o, ci_o, diag, A_or, A_gpu)
+    assert not bad, f"{len(bad)} rows differ beyond boundary and score-error cases, e.g. row " \
+                    f"{bad[0][0]}: gpu {bad[0][1]} oracle {bad[0][2]}"
+    return counts
 
 
 def _check_output(O_gpu, O_ref):
@@ -102,7 +141,9 @@ def test_small_configs_end_to_end(name, w, cuda_device):
     assert np.array_equal(rp, rp_same) and np.array_equal(ci, ci_same)
     # end to end against the oracle's own scores
     rp_o, ci_o, diag = oracle.select(A_or, w.tau, True, diag=True)
-    nb, nm = _check_masks(_csr_rows(rp, ci), rp_o, ci_o, diag)
+    H, Nb = w.H, w.Nb
+    _check_masks(_csr_rows(rp, ci), rp_o, ci_o, diag, A_or.reshape(H * Nb, Nb),
+                 A_gpu.reshape(H * Nb, Nb))
     # output on every row, same CSR on both sides
     rows = [(h, q) for h in range(w.H) for q in range(w.L)]
     if len(rows) > 60000:
@@ -364,33 +405,54 @@ def test_estimate_head_slices(strategy, layer, cuda_device):
     assert np.abs(As.cpu().numpy() - A_or[2:6]).max() <= SCORE_TOL
 
 
-FULL = [(i, workloads.get(i)) for i in (1, 2, 3, 4)]
+FULL = [(i, workloads.get(i)) for i in (0, 1, 2, 3, 4)]
 
 
 @pytest.mark.parametrize("idx,w", FULL, ids=[f"cfg{i}" for i, _ in FULL])
-def test_full_size_sampled(idx, w, cuda_device):
-    """Full-size layers in the benchmark's launch configuration; the oracle recomputes two
-    heads' block scores and masks, and sampled output rows under the GPU's CSR."""
+def test_full_size_layers(idx, w, cuda_device):
+    """The five layers at full size in the benchmark's launch configuration.  Every head:
+    block scores against the oracle; the selection from the GPU's own scores identical to
+    the oracle's on every row; end-to-end masks classified as in the module docstring; then
+    sampled output rows under the GPU's CSR."""
+    import json
+    import os
+
     t = workloads.generate(w)
     d = _to(t, cuda_device)
     A_gpu, rp, ci, O = _gpu_pipeline(w, d, cuda_device)
     del d
-    Nb = w.Nb
-    rng = np.random.default_rng(idx)
-    heads = sorted(rng.choice(w.H, 2, replace=False).tolist())
-    for h in heads:
-        A_or = oracle.estimate(t["Q"], t["K"], w.S, w.B, heads=(h, h + 1))
-        err = np.abs(A_gpu[h].astype(np.float64) - A_or[h]).max()
-        assert err <= SCORE_TOL, f"head {h}: block score error {err:.3e}"
-        rp_o, ci_o, diag = oracle.select(A_or[h:h + 1], w.tau, True, diag=True)
-        gpu_rows = _csr_rows(rp, ci)[h * Nb:(h + 1) * Nb]
-        _check_masks(gpu_rows, rp_o, ci_o, diag)
-    # invariants on every head: rows sum to 1, zero upper triangle, CSR well formed
+    H, Nb = w.H, w.Nb
+    assert rr.validate_csr(torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(), H, Nb) == 0
     assert np.abs(A_gpu.sum(-1) - 1.0).max() < 1e-4
-    assert rr.validate_csr(torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(), w.H, Nb) == 0
+    # the same scores on both sides: identical selection on every row of every head
+    rp_same, ci_same = oracle.select(A_gpu, w.tau, True)
+    assert np.array_equal(rp, rp_same) and np.array_equal(ci, ci_same)
+    # each side from its own scores
+    A_or = oracle.estimate(t["Q"], t["K"], w.S, w.B)
+    err = np.abs(A_gpu.astype(np.float64) - A_or)
+    score_err = float(err.max())
+    assert score_err <= SCORE_TOL, f"block score error {score_err:.3e}"
+    rp_o, ci_o, diag = oracle.select(A_or, w.tau, True, diag=True)
+    counts, bad = _classify_masks(_csr_rows(rp, ci), rp_o, ci_o, diag, A_or.reshape(H * Nb, Nb),
+                                  A_gpu.reshape(H * Nb, Nb))
+    causal = H * Nb * (Nb + 1) // 2
+    record = {"layer": w.name, "H": H, "Hkv": w.Hkv, "L": w.L, "d": w.d, "S": w.S, "B": w.B,
+              "tau": w.tau, "heads_checked": H, **counts, "unexplained": len(bad),
+              "max_score_err": score_err, "same_score_selection_identical": True,
+              "density_gpu": int(rp[-1]) / causal, "density_oracle": int(rp_o[-1]) / causal}
+    print(json.dumps(record))
+    out_dir = os.environ.get("RR_PARITY_RECORD")
+    if out_dir:
+        os.makedirs(out_dir, exist_ok=True)
+        with open(os.path.join(out_dir, f"mask_parity_{w.name}.json"), "w") as f:
+            json.dump(record, f, indent=1)
+    assert not bad, f"{len(bad)} rows differ beyond boundary and score-error cases, e.g. row " \
+                    f"{bad[0][0]}: gpu {bad[0][1]} oracle {bad[0][2]}"
+    del A_or, err
+    rng = np.random.default_rng(idx)
     rows = []
-    for h in range(w.H):
-        for I in [Nb - 1] + rng.choice(Nb, 3, replace=False).tolist():
+    for h in range(H):
+        for I in [Nb - 1] + rng.choice(Nb, min(3, Nb), replace=False).tolist():
             rows += [(h, I * w.B + int(x)) for x in rng.choice(w.B, 2, replace=False)]
         rows += [(h, 0), (h, 1)]
     O_ref = oracle.prefill_rows(t["Q"], t["K"], t["V"], w.B, rp, ci, rows)
@@ -407,13 +469,20 @@ def test_selection_accuracy_diagnostic(cuda_device):
     t = workloads.generate(w)
     d = _to(t, cuda_device)
     res = diagnostics.selection_accuracy(d["Q"], d["K"], w.S, w.B, w.tau)
+    H, Nb = w.H, w.Nb
+    # the masks the diagnostic compares: the oracle's selection from the GPU's scores (identical
+    # to the GPU's on every row), themselves within the mask rules of the oracle's own masks
+    A_rr_gpu = rr.estimate(d["Q"], d["K"], w.S, w.B).cpu().numpy()
+    A_ex_gpu = rr.estimate(d["Q"], d["K"], 1, w.B).cpu().numpy()
     A_rr = oracle.estimate(t["Q"], t["K"], w.S, w.B)
     A_ex = oracle.estimate(t["Q"], t["K"], 1, w.B)
-    rp1, ci1, dg1 = oracle.select(A_rr, w.tau, True, diag=True)
-    rp2, ci2, dg2 = oracle.select(A_ex, w.tau, True, diag=True)
-    if _boundary_rows(dg1).any() or _boundary_rows(dg2).any():
-        pytest.skip("a selection boundary row makes the masks legitimately differ")
-    H, Nb = w.H, w.Nb
+    assert np.abs(A_ex_gpu - A_ex).max() <= SCORE_TOL
+    rp1, ci1 = oracle.select(A_rr_gpu, w.tau, True)
+    rp2, ci2 = oracle.select(A_ex_gpu, w.tau, True)
+    for A_g, A_o, rp_g, ci_g in ((A_rr_gpu, A_rr, rp1, ci1), (A_ex_gpu, A_ex, rp2, ci2)):
+        rp_o, ci_o, dg = oracle.select(A_o, w.tau, True, diag=True)
+        _check_masks(_csr_rows(rp_g, ci_g), rp_o, ci_o, dg, A_o.reshape(H * Nb, Nb),
+                     A_g.reshape(H * Nb, Nb))
     sel = np.zeros((H, Nb, Nb), bool)
     ref = np.zeros((H, Nb, Nb), bool)
     for r in range(H * Nb):
