@@ -4,13 +4,14 @@
 // blocks whose cumulative score reaches tau) with last-query-block protection (Sec. 4.3).
 //
 //   select_rows_warp_kernel  one warp per row of up to 1024 causal blocks: the cut score by a
-//                       binary search over float bit patterns with float64 sums, ties at the
-//                       cut taken in ascending J; selected blocks as a bitmap.
+//                       binary search over float bit patterns with exact 64-bit fixed-point
+//                       sums, ties at the cut taken in ascending J; selected blocks as a bitmap.
 //   select_rows_kernel  one CTA per longer row: bitonic sort of the row's causal scores on the
 //                       key (score desc, J asc), float64 inclusive scan,
 //                       k* = 1 + #{k : cum_k < tau*T}, selected blocks as a bitmap.
 //   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr, nnz.
-//   emit_csr_kernel     one warp per row: bitmap -> ascending block indices in col_idx.
+//   emit_csr_kernel     one warp per row: bitmap -> ascending block indices in col_idx, one
+//                       coalesced store per 32 blocks.
 //   validate_csr_kernel debug check of a CSR, counts bad rows, never traps.
 #include "rr_common.cuh"
 
@@ -135,16 +136,135 @@ __global__ void __launch_bounds__(kSelThreads)
 
 // Warp per row for rows of at most 32*32 blocks (values held in registers, lane l owns blocks
 // J = l + 32*k).  The selected set is the first k* keys in (score desc, J asc) order; it is
-// found without sorting: s* = the largest score with sum_{a >= s*} a >= tau*T (binary search
+// found without sorting: s* = the largest score with sum_{a >= s*} a >= tau*T (a binary search
 // over the bit patterns, which order non-negative floats), then all scores above s* plus the
-// ties at s* in ascending J until the sum reaches tau*T.  Sums in float64.
-__device__ __forceinline__ double warp_sum_d(double v) {
+// ties at s* in ascending J until the sum reaches tau*T.
+//
+// The decision is exact on a 64-bit fixed-point grid: a score is worth its value times
+// 2^(176 - E), E the biased exponent of the row maximum, truncated (a score keeps all 24 bits
+// of its significand when it is within 2^-26 of the maximum, and everything down to 2^-50 of
+// it; the row total stays below 2^60).  T is summed exactly on that grid, tau*T is formed in
+// float64 and rounded up to it, so "cum >= tau*T" is decided exactly, with no dependence on
+// summation order.  Each round of the search first sums in fp32 (one compare and one add per
+// score) and settles the comparison from that sum whenever it is further from tau*T than the
+// fp32 rounding error can reach (37 roundings of 2^-24 relative each; the bound used is 4e-6);
+// only rounds that land closer are re-summed exactly on the grid.  A warp holds its row in
+// NS registers per lane, NS the row's 32-block slots rounded up to a multiple of 4, so short
+// rows do not pay for the longest row's slots.
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Fixed-point value of a non-negative float with bit pattern b, on the grid of a row whose
+// maximum has biased exponent E (E >= 1): b's value times 2^(176 - E), truncated.
+__device__ __forceinline__ long long to_fixed(uint32_t b, int E) {
+    const int e = (int)(b >> 23);
+    const uint32_t m = e ? ((b & 0x7fffffu) | 0x800000u) : (b & 0x7fffffu);
+    const int sh = (e ? e : 1) + 26 - E;  // <= 26: the row maximum's significand lands below 2^50
+    if (sh >= 0) return (long long)m << sh;
+    return sh > -24 ? (long long)(m >> -sh) : 0ll;
+}
+
+template <int NS>
+__device__ __forceinline__ void select_row_warp(const float *__restrict__ a, int n, double tau, int lane,
+                                                uint32_t *__restrict__ out_bm, int W, int *__restrict__ count) {
+    float v[NS];  // scores (-0 as +0); 0 beyond the row
+    uint32_t vmax = 0;
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        const int J = k * 32 + lane;
+        const float x = J < n ? __ldg(a + J) : 0.f;
+        v[k] = (x == 0.f) ? 0.f : x;
+        vmax = max(vmax, __float_as_uint(v[k]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    const int E = max((int)(vmax >> 23), 1);
+    long long tot = 0;
+#pragma unroll
+    for (int k = 0; k < NS; ++k) tot += to_fixed(__float_as_uint(v[k]), E);
+    const long long T = warp_sum_ll(tot);
+    // tau*T rounded up to the grid: for an integer sum c, c >= tau*T <=> c >= thr
+    const long long thr = __double2ll_ru(tau * (double)T);
+    // the same threshold in value units, widened by the fp32 error bound on both sides.  Rows
+    // whose maximum is below 2^-87 (where fp32 sums lose their relative accuracy) and tau below
+    // 1e-4 (where the grid's truncation, up to 2^-39 of the maximum, is no longer far below
+    // the margin) always take the exact sums.
+    const bool fast = E > 40 && tau >= 1e-4;
+    const double thr_val = ldexp((double)thr, E - 176);
+    const float thr_hi = (float)(thr_val * (1.0 + 4e-6)), thr_lo = (float)(thr_val * (1.0 - 4e-6));
+    // largest u in [0, vmax] with sum_{bits(a) >= u} a >= thr (true at u = 0)
+    uint32_t lo = 0, hi = vmax;
+    while (lo < hi) {
+        const uint32_t mid = lo + (hi - lo + 1) / 2;
+        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NS; k += 2) {
+            if (__float_as_uint(v[k]) >= mid) p0 += v[k];
+            if (__float_as_uint(v[k + 1]) >= mid) p1 += v[k + 1];
+        }
+        const float p = warp_sum_f(p0 + p1);
+        bool ge;
+        if (fast && p >= thr_hi) ge = true;
+        else if (fast && p < thr_lo) ge = false;
+        else {
+            long long q = 0;
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                if (__float_as_uint(v[k]) >= mid) q += to_fixed(__float_as_uint(v[k]), E);
+            ge = warp_sum_ll(q) >= thr;
+        }
+        if (ge) lo = mid;
+        else hi = mid - 1;
+    }
+    const uint32_t sbits = lo;
+    long long gt = 0;
+    int cnt_gt = 0;
+#pragma unroll
+    for (int k = 0; k < NS; ++k)
+        if (__float_as_uint(v[k]) > sbits) {
+            gt += to_fixed(__float_as_uint(v[k]), E);
+            ++cnt_gt;
+        }
+    gt = warp_sum_ll(gt);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt_gt += __shfl_xor_sync(0xffffffffu, cnt_gt, o);
+    // ties at s*, ascending J: the smallest t >= 1 with gt + t*s >= thr (gt < thr because s*
+    // is the largest score that reaches the threshold; a zero s* can only mean thr <= gt,
+    // which happens for an all-zero row, where the first block is kept)
+    const long long sfx = to_fixed(sbits, E);
+    long long need_ll = 1;
+    if (sfx > 0 && thr > gt) need_ll = (thr - gt + sfx - 1) / sfx;
+    const int need_ties = (int)min(max(need_ll, 1ll), (long long)(32 * kWarpRowSlots));
+    // emit the bitmap: blocks above s*, plus the first need_ties ties by ascending J
+    int taken = 0;
+    for (int w = NS + lane; w < W; w += 32) out_bm[w] = 0u;
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        const int J = k * 32 + lane;
+        const bool valid = J < n;
+        const uint32_t b = __float_as_uint(v[k]);
+        const bool above = valid && b > sbits;
+        const bool tie = valid && b == sbits;
+        const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+        const int before = __popc(tb & ((1u << lane) - 1u));
+        const bool take_tie = tie && (taken + before < need_ties);
+        taken += __popc(tb);
+        const uint32_t sel = __ballot_sync(0xffffffffu, above || take_tie);
+        if (lane == 0 && k < W) out_bm[k] = sel;  // word k covers blocks 32k..32k+31
+    }
+    if (lane == 0) *count = cnt_gt + min(need_ties, taken);
+}
+
+__global__ void __launch_bounds__(256, 4)
     select_rows_warp_kernel(const float *__restrict__ A, int Nb, long nrows, double tau,
                             int protect_last, int W, int *__restrict__ counts,
                             uint32_t *__restrict__ bitmap) {
@@ -167,86 +287,17 @@ __global__ void __launch_bounds__(256)
         return;
     }
     const float *a = A + row * (long)Nb;
-    const int slots = (n + 31) >> 5;
-    uint32_t v[kWarpRowSlots];  // bit patterns (-0 as +0); 0 beyond the row
-    double tot = 0.0;
-    uint32_t vmax = 0;
-#pragma unroll
-    for (int k = 0; k < kWarpRowSlots; ++k) {
-        v[k] = 0;
-        if (k < slots) {
-            const int J = k * 32 + lane;
-            if (J < n) {
-                const float x = __ldg(a + J);
-                v[k] = (x == 0.f) ? 0u : __float_as_uint(x);
-                tot += (double)x;
-                vmax = max(vmax, v[k]);
-            }
-        }
+    int *cnt = counts + row;
+    switch ((n + 127) >> 7) {  // 32-block slots per lane, rounded up to a multiple of 4
+    case 1: select_row_warp<4>(a, n, tau, lane, out_bm, W, cnt); break;
+    case 2: select_row_warp<8>(a, n, tau, lane, out_bm, W, cnt); break;
+    case 3: select_row_warp<12>(a, n, tau, lane, out_bm, W, cnt); break;
+    case 4: select_row_warp<16>(a, n, tau, lane, out_bm, W, cnt); break;
+    case 5: select_row_warp<20>(a, n, tau, lane, out_bm, W, cnt); break;
+    case 6: select_row_warp<24>(a, n, tau, lane, out_bm, W, cnt); break;
+    case 7: select_row_warp<28>(a, n, tau, lane, out_bm, W, cnt); break;
+    default: select_row_warp<32>(a, n, tau, lane, out_bm, W, cnt); break;
     }
-    const double T = warp_sum_d(tot);
-    const double thr = tau * T;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-    // largest u in [0, vmax] with sum_{bits(a) >= u} a >= thr (true at u = 0)
-    uint32_t lo = 0, hi = vmax;
-    while (lo < hi) {
-        const uint32_t mid = lo + (hi - lo + 1) / 2;
-        double part = 0.0;
-#pragma unroll
-        for (int k = 0; k < kWarpRowSlots; ++k)
-            if (k < slots && v[k] >= mid) part += (double)__uint_as_float(v[k]);
-        if (warp_sum_d(part) >= thr) lo = mid;
-        else hi = mid - 1;
-    }
-    const uint32_t sbits = lo;
-    double gt = 0.0;
-    int cnt_gt = 0;
-#pragma unroll
-    for (int k = 0; k < kWarpRowSlots; ++k)
-        if (k < slots && v[k] > sbits) {
-            gt += (double)__uint_as_float(v[k]);
-            ++cnt_gt;
-        }
-    gt = warp_sum_d(gt);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt_gt += __shfl_xor_sync(0xffffffffu, cnt_gt, o);
-    // ties at s*, ascending J, until the running sum reaches thr (at least one block in all)
-    const double sval = (double)__uint_as_float(sbits);
-    int need_ties = 0;
-    {
-        double run = gt;
-        int take = 0;
-        // count of ties needed: smallest t >= 0 with gt + t*s >= thr (t >= 1 if no block yet)
-        if (!(run >= thr) || cnt_gt == 0) {
-            const double q = (sval > 0.0) ? ceil((thr - run) / sval) : 1.0;
-            take = (int)fmin(fmax(q, 1.0), 32.0 * kWarpRowSlots + 1.0);
-            if (take < 1) take = 1;
-            // guard the division against rounding: step until the sum rule holds exactly
-            while (take > 1 && run + (double)(take - 1) * sval >= thr) --take;
-            while (run + (double)take * sval < thr) ++take;
-        }
-        need_ties = take;
-    }
-    // emit the bitmap: blocks above s*, plus the first need_ties ties by ascending J
-    int taken = 0;
-    for (int w = lane; w < W; w += 32) out_bm[w] = 0u;
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < kWarpRowSlots; ++k) {
-        if (k >= slots) break;
-        const int J = k * 32 + lane;
-        const bool valid = J < n;
-        const bool above = valid && v[k] > sbits;
-        const bool tie = valid && v[k] == sbits;
-        const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-        const int before = __popc(tb & ((1u << lane) - 1u));
-        const bool take_tie = tie && (taken + before < need_ties);
-        taken += __popc(tb);
-        const uint32_t sel = __ballot_sync(0xffffffffu, above || take_tie);
-        if (lane == 0) out_bm[k] = sel;  // W >= slots; word k covers blocks 32k..32k+31
-    }
-    if (lane == 0) counts[row] = cnt_gt + min(need_ties, taken);
 }
 
 __global__ void __launch_bounds__(1024)
@@ -292,25 +343,18 @@ __global__ void __launch_bounds__(256)
     const int lane = threadIdx.x & 31;
     if (row >= nrows) return;
     const uint32_t *bm = bitmap + row * W;
+    const uint32_t below = (1u << lane) - 1u;
     int at = row_ptr[row];
     for (int w0 = 0; w0 < W; w0 += 32) {
-        const int w = w0 + lane;
-        const uint32_t m = (w < W) ? bm[w] : 0u;
-        const int c = __popc(m);
-        int x = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+        const uint32_t mine = (w0 + lane < W) ? bm[w0 + lane] : 0u;
+        const int nw = min(32, W - w0);
+        // word k covers blocks 32(w0+k) .. +31: lane l stores block 32(w0+k)+l if its bit is set,
+        // at the position counted by the set bits below it, so the warp's stores are contiguous
+        for (int k = 0; k < nw; ++k) {
+            const uint32_t m = __shfl_sync(0xffffffffu, mine, k);
+            if (m >> lane & 1u) col_idx[at + __popc(m & below)] = (w0 + k) * 32 + lane;
+            at += __popc(m);
         }
-        int pos = at + x - c;
-        uint32_t mm = m;
-        while (mm) {
-            const int b = __ffs(mm) - 1;
-            col_idx[pos++] = w * 32 + b;
-            mm &= mm - 1;
-        }
-        at += __shfl_sync(0xffffffffu, x, 31);
     }
 }
 
