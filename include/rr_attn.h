@@ -110,8 +110,11 @@ size_t rr_select_workspace_bytes(int H, int Nb);
  * For every head h and query block I (row r = h*Nb + I) the causal scores
  * block_scores[h][I][0..I] are ordered by (score descending, J ascending); with T the row
  * total and cum_k the sum of the first k, the row keeps the first k* blocks where k* is the
- * smallest k with cum_k >= tau * T.  Sums and the comparison are in float64.  tau >= 1, or
- * protect_last != 0 and I = Nb-1, keeps all I+1 blocks.  Every row keeps at least 1 block.
+ * smallest k with cum_k >= tau * T.  Precision of the decision: for rows of up to 1024
+ * blocks the sums are exact integers on a fixed-point grid set by the row maximum (every
+ * score keeps its bits down to 2^-50 of the maximum) and tau * T is formed in float64 and
+ * rounded up to that grid; longer rows sum in float64.  tau >= 1, or protect_last != 0 and
+ * I = Nb-1, keeps all I+1 blocks.  Every row keeps at least 1 block.
  *
  * Output (device, caller-owned): row_ptr int32 [H*Nb + 1] (row_ptr[0] = 0) and col_idx
  * int32 [col_capacity]; row r's blocks are col_idx[row_ptr[r] .. row_ptr[r+1]) in strictly
@@ -136,7 +139,8 @@ rr_status_t rr_select(const float *block_scores, int H, int Nb, double tau, int 
  * Scratch: a fixed 8 MiB array compiled into the library (held by every GPU that loads it
  * until the process exits).  Sizes with rr_select_workspace_bytes(H, Nb) > 8 MiB are rejected
  * with RR_ERR_UNSUPPORTED before any launch.  The first call on a device (with that device
- * current) looks up the array's device address once; make it before any stream capture.
+ * current) looks up the array's device address and keeps it; make it before any stream
+ * capture.  If that lookup fails the call returns RR_ERR_CUDA and the next call retries it.
  * All calls share the array: calls that overlap on the GPU (unordered streams or threads)
  * race; each call writes every scratch word it reads, so no clearing is needed.
  */

@@ -7,6 +7,13 @@
 
 #include "rr_common.cuh"
 
+// NVTX ranges around the entry points (header-only NVTX 3; a profiler that injects NVTX, such
+// as Nsight Systems, shows them on the host timeline, otherwise they cost a branch each).
+#if __has_include(<nvtx3/nvToolsExt.h>)
+#include <nvtx3/nvToolsExt.h>
+#define RR_NVTX 1
+#endif
+
 namespace rr {
 
 size_t estimate_workspace_bytes(int Hkv, int L, int d, int S);
@@ -25,7 +32,14 @@ rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16
                               float scale, uint16_t *O, cudaStream_t st);
 rr_status_t read_device_errors(unsigned *out, bool reset);
 rr_status_t read_estimate_errors(unsigned *out, bool reset);
+rr_status_t read_pp_errors(unsigned *out, bool reset);
 rr_status_t selftest_wait(uint32_t timeout_us, uint32_t *result);
+
+#define RR_TRY(x)                       \
+    do {                                \
+        const rr_status_t s_ = (x);     \
+        if (s_ != RR_OK) return s_;     \
+    } while (0)
 
 static thread_local char g_last_error[512] = "";
 
@@ -37,16 +51,61 @@ rr_status_t set_error(rr_status_t s, const char *fmt, ...) {
     return s;
 }
 
+void clear_error() { g_last_error[0] = 0; }
+
+rr_status_t check_ptr(const char *fn, const char *name, const void *p) {
+    if (!p) return set_error(RR_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);
+    if (!aligned16(p)) return set_error(RR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, name);
+    return RR_OK;
+}
+
 rr_status_t check_launch(const char *what) {
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(RR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return RR_OK;
 }
 
+rr_status_t check_select_args(const char *fn, const float *block_scores, int H, int Nb, double tau,
+                              const int32_t *row_ptr, const int32_t *col_idx, int64_t col_capacity,
+                              const int64_t *nnz_out) {
+    if (H <= 0 || Nb < 0 || H > kMaxH || Nb > kMaxL / 64)
+        return set_error(RR_ERR_INVALID_ARG, "%s: bad sizes H=%d Nb=%d", fn, H, Nb);
+    if (!(tau > 0.0 && tau <= 1.0) || std::isnan(tau))
+        return set_error(RR_ERR_INVALID_ARG, "%s: tau=%g must be in (0, 1]", fn, tau);
+    if (Nb == 0) return RR_OK;
+    const int64_t worst = (int64_t)H * Nb * (Nb + 1) / 2;
+    if (worst > INT32_MAX)
+        return set_error(RR_ERR_UNSUPPORTED, "%s: worst-case nnz %lld exceeds int32", fn, (long long)worst);
+    if (col_capacity < worst)
+        return set_error(RR_ERR_INVALID_ARG, "%s: col_capacity %lld < worst case %lld", fn,
+                         (long long)col_capacity, (long long)worst);
+    RR_TRY(check_ptr(fn, "block_scores", block_scores));
+    RR_TRY(check_ptr(fn, "row_ptr", row_ptr));
+    RR_TRY(check_ptr(fn, "col_idx", col_idx));
+    if (nnz_out && (reinterpret_cast<uintptr_t>(nnz_out) & 7))
+        return set_error(RR_ERR_INVALID_ARG, "%s: nnz_out is not 8-byte aligned", fn);
+    return RR_OK;
+}
+
 namespace {
 
-constexpr int kMaxL = 1 << 20;
-constexpr int kMaxH = 256;
+// Scoped NVTX range named after the entry point.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) {
+#ifdef RR_NVTX
+        nvtxRangePushA(name);
+#else
+        (void)name;
+#endif
+    }
+    ~NvtxRange() {
+#ifdef RR_NVTX
+        nvtxRangePop();
+#endif
+    }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 rr_status_t check_common(const char *fn, int H, int Hkv, int L, int d, int B) {
     if (H <= 0 || Hkv <= 0 || L < 0 || d <= 0 || B <= 0)
@@ -64,18 +123,6 @@ rr_status_t check_common(const char *fn, int H, int Hkv, int L, int d, int B) {
         return set_error(RR_ERR_UNSUPPORTED, "%s: L=%d or H=%d above the supported maximum", fn, L, H);
     return RR_OK;
 }
-
-rr_status_t check_ptr(const char *fn, const char *name, const void *p) {
-    if (!p) return set_error(RR_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);
-    if (!aligned16(p)) return set_error(RR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, name);
-    return RR_OK;
-}
-
-#define RR_TRY(x)                       \
-    do {                                \
-        const rr_status_t s_ = (x);     \
-        if (s_ != RR_OK) return s_;     \
-    } while (0)
 
 }  // namespace
 }  // namespace rr
@@ -100,17 +147,18 @@ const char *rr_status_string(rr_status_t s) {
 const char *rr_last_error(void) { return g_last_error; }
 
 rr_status_t rr_device_errors(uint32_t *flags, int reset) {
-    g_last_error[0] = 0;
+    clear_error();
     if (!flags) return set_error(RR_ERR_INVALID_ARG, "rr_device_errors: flags is NULL");
-    unsigned v = 0, ve = 0;
+    unsigned v = 0, ve = 0, vp = 0;
     rr_status_t s = read_device_errors(&v, reset != 0);
     if (s == RR_OK) s = read_estimate_errors(&ve, reset != 0);
-    *flags = v | ve;
+    if (s == RR_OK) s = read_pp_errors(&vp, reset != 0);
+    *flags = v | ve | vp;
     return s;
 }
 
 rr_status_t rr_selftest_wait(uint32_t timeout_us, uint32_t *result) {
-    g_last_error[0] = 0;
+    clear_error();
     if (!result) return set_error(RR_ERR_INVALID_ARG, "rr_selftest_wait: result is NULL");
     if (timeout_us == 0 || timeout_us > 2000000u)
         return set_error(RR_ERR_INVALID_ARG, "rr_selftest_wait: timeout_us=%u outside (0, 2e6]",
@@ -130,7 +178,8 @@ rr_status_t rr_estimate_heads(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int
                               float *block_scores, void *workspace, size_t workspace_bytes,
                               rr_stream_t stream) {
     static const char *fn = "rr_estimate";
-    g_last_error[0] = 0;
+    const NvtxRange range(fn);
+    clear_error();
     RR_TRY(check_common(fn, H, Hkv, L, d, B));
     if (S <= 0 || S > B || B % S)
         return set_error(RR_ERR_INVALID_ARG, "%s: stride S=%d must divide B=%d", fn, S, B);
@@ -179,23 +228,10 @@ rr_status_t rr_select(const float *block_scores, int H, int Nb, double tau, int 
                       int64_t *nnz_out, void *workspace, size_t workspace_bytes,
                       rr_stream_t stream) {
     static const char *fn = "rr_select";
-    g_last_error[0] = 0;
-    if (H <= 0 || Nb < 0 || H > kMaxH || Nb > kMaxL / 64)
-        return set_error(RR_ERR_INVALID_ARG, "%s: bad sizes H=%d Nb=%d", fn, H, Nb);
-    if (!(tau > 0.0 && tau <= 1.0) || std::isnan(tau))
-        return set_error(RR_ERR_INVALID_ARG, "%s: tau=%g must be in (0, 1]", fn, tau);
+    const NvtxRange range(fn);
+    clear_error();
+    RR_TRY(check_select_args(fn, block_scores, H, Nb, tau, row_ptr, col_idx, col_capacity, nnz_out));
     if (Nb == 0) return RR_OK;
-    const int64_t worst = (int64_t)H * Nb * (Nb + 1) / 2;
-    if (worst > INT32_MAX)
-        return set_error(RR_ERR_UNSUPPORTED, "%s: worst-case nnz %lld exceeds int32", fn, (long long)worst);
-    if (col_capacity < worst)
-        return set_error(RR_ERR_INVALID_ARG, "%s: col_capacity %lld < worst case %lld", fn,
-                         (long long)col_capacity, (long long)worst);
-    RR_TRY(check_ptr(fn, "block_scores", block_scores));
-    RR_TRY(check_ptr(fn, "row_ptr", row_ptr));
-    RR_TRY(check_ptr(fn, "col_idx", col_idx));
-    if (nnz_out && (reinterpret_cast<uintptr_t>(nnz_out) & 7))
-        return set_error(RR_ERR_INVALID_ARG, "%s: nnz_out is not 8-byte aligned", fn);
     const size_t need = select_workspace_bytes(H, Nb);
     if (!workspace || workspace_bytes < need)
         return set_error(RR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
@@ -210,7 +246,8 @@ rr_status_t rr_sparse_prefill(const rr_bf16_t *Q, const rr_bf16_t *K, const rr_b
                               const int32_t *col_idx, float softmax_scale, rr_bf16_t *O,
                               rr_stream_t stream) {
     static const char *fn = "rr_sparse_prefill";
-    g_last_error[0] = 0;
+    const NvtxRange range(fn);
+    clear_error();
     RR_TRY(check_common(fn, H, Hkv, L, d, B));
     if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
         return set_error(RR_ERR_INVALID_ARG, "%s: softmax_scale is not finite", fn);
@@ -229,7 +266,7 @@ rr_status_t rr_sparse_prefill(const rr_bf16_t *Q, const rr_bf16_t *K, const rr_b
 rr_status_t rr_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int H, int Nb,
                             int64_t nnz_cap, int32_t *bad_rows, rr_stream_t stream) {
     static const char *fn = "rr_validate_csr";
-    g_last_error[0] = 0;
+    clear_error();
     if (H <= 0 || Nb <= 0 || nnz_cap < 0)
         return set_error(RR_ERR_INVALID_ARG, "%s: bad sizes", fn);
     RR_TRY(check_ptr(fn, "row_ptr", row_ptr));

@@ -11,8 +11,23 @@ namespace rr {
 // ---------------------------------------------------------------- host-side errors
 rr_status_t set_error(rr_status_t s, const char *fmt, ...);
 rr_status_t check_launch(const char *what);
+// Empties the calling thread's last-error text; every entry point calls it first.
+void clear_error();
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Largest sizes any entry point accepts.
+constexpr int kMaxL = 1 << 20;
+constexpr int kMaxH = 256;
+
+// Non-null and 16-byte aligned, else RR_ERR_INVALID_ARG with the argument's name.
+rr_status_t check_ptr(const char *fn, const char *name, const void *p);
+
+// The host-side checks of rr_select's arguments other than its workspace (sizes, tau, the
+// output capacity, pointers), shared by every selection entry point.
+rr_status_t check_select_args(const char *fn, const float *block_scores, int H, int Nb, double tau,
+                              const int32_t *row_ptr, const int32_t *col_idx, int64_t col_capacity,
+                              const int64_t *nnz_out);
 
 // TMA descriptor (a CUtensorMap, 128 bytes, 64-byte aligned) of a 2-D row-major bf16 tensor
 // [rows][cols]: boxes of 64 columns x box_rows rows, 128-byte swizzle.  False when the

@@ -446,12 +446,16 @@ rr_status_t launch_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, i
 
 }  // namespace
 
+rr_status_t launch_prefill_pp(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H, int Hkv,
+                              int L, int d, const int32_t *row_ptr, const int32_t *col_idx, float scale,
+                              uint16_t *O, cudaStream_t st);
+
+// B = 128: two query tiles per CTA (rr_prefill_pp.cu); B = 64: this file's one-tile kernel.
 rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int H, int Hkv,
                               int L, int d, int B, const int32_t *row_ptr, const int32_t *col_idx,
                               float scale, uint16_t *O, cudaStream_t st) {
-    if (d == 128 && B == 128) return launch_tc<128, 128>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
-    if (d == 128 && B == 64) return launch_tc<128, 64>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
-    if (d == 64 && B == 128) return launch_tc<64, 128>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
+    if (B == 128) return launch_prefill_pp(Q, K, V, H, Hkv, L, d, row_ptr, col_idx, scale, O, st);
+    if (d == 128) return launch_tc<128, 64>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
     return launch_tc<64, 64>(Q, K, V, H, Hkv, L, row_ptr, col_idx, scale, O, st);
 }
 

@@ -13,7 +13,8 @@
 // Set-up: the first call on a device, with that device current, looks up the array's device
 // address with cudaGetSymbolAddress (a host-side name of a __device__ array is only a stand-in,
 // never a usable device pointer) and caches it for that device.  Make that first call on each
-// device before any stream capture begins.
+// device before any stream capture begins.  Only a successful lookup is cached: a failed one
+// returns RR_ERR_CUDA and the next call on that device tries again.
 //
 // Sharing: all calls on a device use the same array and it keeps whatever the last call left.
 // Every word a call reads is first written by the same call (each row writes its count and all
@@ -38,9 +39,22 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
-void *g_scratch_addr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxDevices];  // the array's device address per device, once looked up
+
+// Device address of the scratch array on the current device `dev` (cached after the first
+// successful lookup), or the CUDA error of the lookup.
+cudaError_t scratch_address(int dev, void **addr) {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return cudaSuccess;
+}
 
 }  // namespace
 
@@ -51,24 +65,11 @@ extern "C" rr_status_t rr_select_noalloc(const float *block_scores, int H, int N
                                          int64_t col_capacity, int64_t *nnz_out,
                                          rr_stream_t stream) {
     static const char *fn = "rr_select_noalloc";
-    if (H <= 0 || Nb < 0 || H > 256 || Nb > (1 << 20) / 64)
-        return set_error(RR_ERR_INVALID_ARG, "%s: bad sizes H=%d Nb=%d", fn, H, Nb);
-    if (!(tau > 0.0 && tau <= 1.0))
-        return set_error(RR_ERR_INVALID_ARG, "%s: tau=%g must be in (0, 1]", fn, tau);
+    clear_error();
+    const rr_status_t st = check_select_args(fn, block_scores, H, Nb, tau, row_ptr, col_idx,
+                                             col_capacity, nnz_out);
+    if (st != RR_OK) return st;
     if (Nb == 0) return RR_OK;
-    const int64_t worst = (int64_t)H * Nb * (Nb + 1) / 2;
-    if (worst > INT32_MAX)
-        return set_error(RR_ERR_UNSUPPORTED, "%s: worst-case nnz %lld exceeds int32", fn,
-                         (long long)worst);
-    if (col_capacity < worst)
-        return set_error(RR_ERR_INVALID_ARG, "%s: col_capacity %lld < worst case %lld", fn,
-                         (long long)col_capacity, (long long)worst);
-    if (!block_scores || !aligned16(block_scores) || !row_ptr || !aligned16(row_ptr) || !col_idx ||
-        !aligned16(col_idx))
-        return set_error(RR_ERR_INVALID_ARG, "%s: block_scores, row_ptr and col_idx must be "
-                                             "non-null and 16-byte aligned", fn);
-    if (nnz_out && (reinterpret_cast<uintptr_t>(nnz_out) & 7))
-        return set_error(RR_ERR_INVALID_ARG, "%s: nnz_out is not 8-byte aligned", fn);
     const size_t need = select_workspace_bytes(H, Nb);
     if (need > kNoAllocScratchBytes)
         return set_error(RR_ERR_UNSUPPORTED,
@@ -81,12 +82,11 @@ extern "C" rr_status_t rr_select_noalloc(const float *block_scores, int H, int N
         return set_error(RR_ERR_CUDA, "%s: cudaGetDevice: %s", fn, cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDevices)
         return set_error(RR_ERR_UNSUPPORTED, "%s: device index %d out of range", fn, dev);
-    std::call_once(g_scratch_once[dev], [dev] {
-        g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], g_select_scratch);
-    });
-    if (g_scratch_err[dev] != cudaSuccess || !g_scratch_addr[dev])
+    void *scratch = nullptr;
+    e = scratch_address(dev, &scratch);
+    if (e != cudaSuccess)
         return set_error(RR_ERR_CUDA, "%s: cudaGetSymbolAddress of the scratch array: %s", fn,
-                         cudaGetErrorString(g_scratch_err[dev]));
+                         cudaGetErrorString(e));
     return launch_select(block_scores, H, Nb, tau, protect_last, row_ptr, col_idx, nnz_out,
-                         g_scratch_addr[dev], static_cast<cudaStream_t>(stream));
+                         scratch, static_cast<cudaStream_t>(stream));
 }

@@ -3,9 +3,11 @@
 Such callers (a plugin whose host application owns all device memory, or a path that must
 never call cudaMalloc/cudaFree) get their scratch from a fixed array inside the library.
 This file is collected last so that a failure here leaves every other test already run.
-It checks the allocation-free call through the C ABI against rr_select on two calls in a row
-with different shapes, so leftovers of the first call in the shared array cannot hide, and
-that sizes beyond the array are refused before any launch.
+It checks the allocation-free call through the C ABI against rr_select on three calls in a
+row with different shapes, so leftovers of an earlier call in the shared array cannot hide;
+the third has rows longer than 1024 blocks, which take the sorting kernel.  It also checks
+that sizes beyond the array are refused before any launch, and that a successful call leaves
+no stale error text behind.
 """
 import ctypes
 
@@ -40,9 +42,11 @@ def _noalloc(A, tau, protect):
     return rp, ci, nnz
 
 
-@pytest.mark.parametrize("first,second", [((32, 256, 0.9, True), (8, 700, 0.8, False))])
-def test_noalloc_matches_select_on_two_calls(first, second, cuda_device):
-    for i, (H, Nb, tau, protect) in enumerate((first, second)):
+CALLS = [(32, 256, 0.9, True), (8, 700, 0.8, False), (2, 1100, 0.9, False)]
+
+
+def test_noalloc_matches_select_on_consecutive_calls(cuda_device):
+    for i, (H, Nb, tau, protect) in enumerate(CALLS):
         A = _scores(H, Nb, seed=i, ties=(i == 1))
         rp_ref, ci_ref, nnz_ref = rr.select(A, tau, protect)
         rp, ci, nnz = _noalloc(A, tau, protect)
@@ -60,3 +64,10 @@ def test_noalloc_refuses_sizes_beyond_the_array(cuda_device):
                                       H * Nb * (Nb + 1) // 2, None, None)
     assert code == 2
     assert b"built-in array" in rr.lib().rr_last_error()
+
+
+def test_noalloc_success_clears_the_last_error(cuda_device):
+    code = rr.lib().rr_select_noalloc(None, 2, 8, 0.9, 1, None, None, 72, None, None)
+    assert code == 1 and rr.lib().rr_last_error() != b""
+    _noalloc(_scores(2, 8, seed=5), 0.9, True)
+    assert rr.lib().rr_last_error() == b""
