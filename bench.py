@@ -47,27 +47,34 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def prefill_traffic_per_launch(w):
-    """DRAM bytes per prefill launch from the committed ncu summary of the 32K Llama-shaped
-    layer, scaled by L (Q, K, V and O all grow linearly with L at fixed heads and d).  None
-    when the kernel source changed since the capture or the layer shape differs."""
+def profile_record(name):
+    """The committed counter record ``profiles/<name>.json`` of one kernel (written from an
+    ncu capture), or None.  It carries the sha256 (first 16 hex digits) of every source the
+    kernel is built from; the record is stale, and None is returned, when any differs now."""
     import hashlib
-    import re
 
-    summ = os.path.join(ROOT, "profiles", "prefill_tc_llama3-8b-layer-L32k.md")
-    src = os.path.join(ROOT, "long_context_prefill_estimate_b200", "csrc", "rr_prefill_tc.cu")
-    if not (os.path.exists(summ) and os.path.exists(src)):
+    path = os.path.join(ROOT, "profiles", name + ".json")
+    if not os.path.exists(path):
         return None
-    text = open(summ).read()
-    m = re.search(r"prefill source sha256: ([0-9a-f]{16})", text)
-    rd = re.search(r"dram__bytes_read.sum / write.sum \| ([0-9.]+) MB / ([0-9.]+) MB", text)
-    if not (m and rd):
+    with open(path) as f:
+        rec = json.load(f)
+    for src, digest in rec.get("sources", {}).items():
+        full = os.path.join(ROOT, src)
+        if not os.path.exists(full) or hashlib.sha256(open(full, "rb").read()).hexdigest()[:16] != digest:
+            return None
+    return rec
+
+
+def prefill_traffic_per_launch(w):
+    """DRAM bytes (read + write) per prefill launch from the committed capture, scaled by L
+    from the captured layer to this one (Q, K, V and O all grow linearly with L at fixed heads
+    and d).  None when the kernel changed since the capture or the layer shape differs."""
+    rec = profile_record("prefill_tc_llama3-8b-layer-L32k")
+    if rec is None:
         return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != m.group(1):
+    if (w.H, w.Hkv, w.d, w.B) != tuple(rec["shape"][k] for k in ("H", "Hkv", "d", "B")):
         return None
-    if (w.H, w.Hkv, w.d, w.B) != (32, 8, 128, 128):
-        return None
-    return (float(rd.group(1)) + float(rd.group(2))) * 1e6 * w.L / 32768
+    return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * w.L / rec["shape"]["L"]
 
 
 def max_over_ranks(value: float, device=None) -> float:
@@ -147,27 +154,27 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_sample(w, t, n_rows: int, rng_seed: int = 0, n_est_heads: int = 1):
-    """Time the oracle on the estimate + select of query heads 0..n_est_heads-1 and on n_rows
-    prefill rows of head 0; extrapolate linearly to the whole layer.
-    Returns (layer_seconds, info)."""
+def oracle_sample(w, t, head: int, n_rows: int, seed: int):
+    """One bounded sample of the oracle on the layer: the estimate and selection of query head
+    `head` (all of its query blocks) and n_rows random prefill rows of that head under its
+    selection, extrapolated linearly to the layer's H heads (the prefill part scaled by the keys
+    attended by all rows of the head over the keys attended by the sampled rows).
+    Returns (layer_seconds, seconds_measured, (A, row_ptr, col_idx, diag) of the head)."""
     import oracle
 
-    h = 0
+    h = head
+    g = h // (w.H // w.Hkv)
     t0 = time.perf_counter()
-    A = oracle.estimate(t["Q"], t["K"], w.S, w.B, heads=(0, n_est_heads))
+    A = oracle.estimate(t["Q"], t["K"], w.S, w.B, heads=(h, h + 1))[h:h + 1]
     t1 = time.perf_counter()
-    rp, ci = oracle.select(A[h:h + 1], w.tau, True)
+    rp, ci, dg = oracle.select(A, w.tau, True, diag=True)
     t2 = time.perf_counter()
-    rng = np.random.default_rng(rng_seed)
+    rng = np.random.default_rng(seed)
     qs = np.sort(rng.choice(w.L, n_rows, replace=False))
-    # the head-0 CSR is rows 0..Nb-1 of a one-head CSR: run the oracle on head 0 alone
     rows = [(0, int(q)) for q in qs]
-    oracle.prefill_rows(t["Q"][h:h + 1], t["K"][:1], t["V"][:1], w.B, rp, ci, rows)
+    oracle.prefill_rows(t["Q"][h:h + 1], t["K"][g:g + 1], t["V"][g:g + 1], w.B, rp, ci, rows)
     t3 = time.perf_counter()
-    est, sel, pre = (t1 - t0) / n_est_heads, t2 - t1, t3 - t2
-    # prefill cost grows with the number of attended keys: scale the sampled rows' time by
-    # (keys attended by all rows of the head) / (keys attended by the sampled rows)
+    est, sel, pre = t1 - t0, t2 - t1, t3 - t2
     B = w.B
     n_off = np.zeros(w.Nb, np.int64)
     has_diag = np.zeros(w.Nb, bool)
@@ -179,9 +186,14 @@ def oracle_sample(w, t, n_rows: int, rng_seed: int = 0, n_est_heads: int = 1):
     Iq = qs // B
     keys_sample = float((n_off[Iq] * B + has_diag[Iq] * (qs - Iq * B + 1)).sum())
     layer = w.H * (est + sel + pre * keys_all / max(keys_sample, 1.0))
-    info = {"estimate_s_per_head": est, "select_s_per_head": sel, "prefill_s_sample": pre,
-            "rows": n_rows, "seconds_measured": t3 - t0}
-    return layer, info
+    return layer, t3 - t0, (A[0], rp, ci, dg)
+
+
+def sample_text(w, n_rows):
+    return (f"per sample: the oracle's estimate and selection of one query head (all {w.Nb} query "
+            f"blocks) and {n_rows} random prefill rows of that head, extrapolated linearly to {w.H} "
+            f"heads and {w.L} rows (the prefill part scaled by attended keys); value from the "
+            f"median sample")
 
 
 # ---------------------------------------------------------------------------- reference arm
@@ -195,24 +207,25 @@ def run_reference(args):
     if args.L:
         w = w.with_(L=args.L)
     t = workloads.generate(w)
-    times = []
-    info = None
+    layer, measured = [], []
     for i in range(args.warmup + args.steps):
-        layer_s, info = oracle_sample(w, t, n_rows=args.ref_rows, rng_seed=i)
+        layer_s, meas_s, _ = oracle_sample(w, t, head=i % w.H, n_rows=args.ref_rows, seed=i)
         if i >= args.warmup:
-            times.append(layer_s)
-    ms = 1e3 * statistics.median(times)
-    val = dense_causal_flops(w) / (ms * 1e-3) / 1e12
-    sample = (f"per step: oracle estimate+select of query head 0 (all {w.Nb} query blocks) and "
-              f"{args.ref_rows} prefill rows of head 0; extrapolated linearly to {w.H} heads and "
-              f"{w.L} rows (prefill scaled by attended keys)")
+            layer.append(layer_s)
+            measured.append(meas_s)
+    layer_ms = 1e3 * statistics.median(layer)
+    val = dense_causal_flops(w) / (layer_ms * 1e-3) / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        # the time one step (one bounded sample) actually took; the layer time it stands for is
+        # extrapolated from it
+        "ms_per_step": 1e3 * statistics.median(measured),
+        "ms_per_layer_extrapolated": layer_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(w, world),
         "cpu_baseline": {"kind": "oracle", "value": val, "unit": "TFLOP/s",
-                         "cores": oracle.threads(), "sample": sample, "last_step": info},
+                         "cores": oracle.threads(), "sample": sample_text(w, args.ref_rows)},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -322,6 +335,8 @@ def run_ours(args):
     rp = ws.row_ptr.cpu().numpy()
     nnz = int(rp[-1])
     ci = ws.col_idx[:nnz].cpu().numpy()
+    A_sample = ws.block_scores[:min(args.cpu_samples, wl.H)].cpu().numpy() \
+        if rank == 0 and not args.no_cpu_baseline else None
     sel_flops, n_diag, n_off = selected_flops(rp, ci, wl.H, wl.Nb, wl.B, wl.d)
     causal_blocks = wl.H * wl.Nb * (wl.Nb + 1) // 2
     dense = dense_causal_flops(w)
@@ -383,17 +398,33 @@ def run_ours(args):
         line["dense_reference"] = dense_comparison(wl, Q, K, V, ws, rr, torch, st, ms_step)
     line["e2e"] = e2e(w, wl, host, h0, layers, rr, torch, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
-        layer_s, info = oracle_sample(w, full, n_rows=args.cpu_rows, n_est_heads=args.cpu_heads)
         import oracle
+        from long_context_prefill_estimate_b200 import diagnostics
 
+        heads = [i % wl.H for i in range(args.cpu_samples)]
+        layer, measured, counts = [], 0.0, None
+        gpu_rows = diagnostics.csr_rows(rp, ci)
+        for i, h in enumerate(heads):
+            layer_s, meas_s, (A_o, rp_o, ci_o, dg_o) = oracle_sample(wl, host, h, args.ref_rows, seed=i)
+            layer.append(layer_s)
+            measured += meas_s
+            if i < wl.H:  # masks of each sampled head against the GPU's (boundary rule 1e-4)
+                c, bad = diagnostics.classify_masks(gpu_rows[h * wl.Nb:(h + 1) * wl.Nb],
+                                                    diagnostics.csr_rows(rp_o, ci_o), dg_o, A_o,
+                                                    A_sample[h])
+                c["unexplained"] = len(bad)
+                counts = c if counts is None else {k: counts[k] + c[k] for k in c}
+        layer_s = statistics.median(layer)
         line["cpu_baseline"] = {
-            "value": dense / layer_s / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": (f"oracle estimate of query heads 0..{args.cpu_heads - 1} (all {w.Nb} query "
-                       f"blocks each), select of head 0 and {args.cpu_rows} random prefill rows of "
-                       f"head 0, extrapolated linearly to the layer ({layer_s:.1f} s/layer); "
-                       f"measured {info['seconds_measured']:.1f} s"),
+            "value": dense / layer_s / 1e12 * (1 if args.shard == "replicas" else wl.H / w.H),
+            "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": sample_text(wl, args.ref_rows) + f"; {len(heads)} samples, "
+                      f"{measured:.1f} s measured",
         }
+        line["mask_parity"] = {**counts, "heads": sorted(set(heads)),
+                               "rule": "GPU vs oracle masks of the sampled heads, each side "
+                                       "from its own scores; boundary = oracle cum within 1e-4 "
+                                       "of tau*T (all heads: profiles/mask_parity_full_size.json)"}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -466,9 +497,9 @@ def e2e(w, wl, host, h0, layers, rr, torch, dev, args):
     st = torch.cuda.current_stream(dev)
     run = lambda: rr.prefill(pinned["Q"], pinned["K"], pinned["V"], w.S, w.B, w.tau, out=out,
                              head_base=h0)
-    for _ in range(max(1, min(args.warmup, 2))):
+    for _ in range(max(1, args.warmup)):
         run()
-    n = max(1, min(args.steps, 5))
+    n = max(1, args.steps)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
@@ -496,9 +527,10 @@ def main(argv=None):
     ap.add_argument("--L", type=int, default=0, help="override the sequence length")
     ap.add_argument("--quick", action="store_true", help="skip the tau sweep and dense comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=8192)
-    ap.add_argument("--cpu-heads", type=int, default=4)
-    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--cpu-samples", type=int, default=12,
+                    help="oracle samples (one query head each) of the CPU baseline")
+    ap.add_argument("--ref-rows", type=int, default=1024,
+                    help="prefill rows per oracle sample (CPU baseline and reference arm)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="replicas: one independent layer per GPU (weak scaling); heads: one "
                          "layer split across the GPUs by whole KV groups (strong scaling)")

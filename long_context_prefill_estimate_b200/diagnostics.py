@@ -53,6 +53,60 @@ def mask_metrics(sel: np.ndarray, ref: np.ndarray, ref_mass: np.ndarray) -> Dict
     return {"precision": precision, "recall": recall, "f1": f1, "captured_mass": captured}
 
 
+def classify_masks(rows_a, rows_b, diag_b, A_b, A_a, cum_tol: float = 1e-4):
+    """Compare two Top-tau selections of the same rows, row by row.
+
+    rows_a, rows_b: per-row lists of selected blocks (ascending) of side a (e.g. the GPU) and
+    side b (a reference selecting from its own scores A_b); row r is query block r % Nb of a
+    head (the lists start at a head boundary).  diag_b: side b's per-row selection record
+    [k*, cum_(k*-1), cum_(k*), tau*T, gap].  A_a, A_b: the two sides' scores of the same
+    rows, [rows][Nb].  A mismatching row is
+      boundary          if side b's cumulative sum just before or at the cut is within
+                        cum_tol of tau*T;
+      near tie          if both keep the same number of blocks and every block they disagree
+                        on has a side-b score within 2*delta of side b's cut score, delta the
+                        row's largest score difference (a score error of delta can swap only
+                        such blocks);
+      sum within error  if the counts differ and a cumulative sum at the cut is within
+                        2*n*delta of tau*T (n causal blocks in the row);
+    and unexplained otherwise.  Returns (counts, unexplained [(row, a, b), ...])."""
+    Nb = np.shape(A_b)[-1]
+    diag_b = np.asarray(diag_b)
+    bnd = (np.abs(diag_b[:, 1] - diag_b[:, 3]) < cum_tol) | (np.abs(diag_b[:, 2] - diag_b[:, 3]) < cum_tol)
+    out = {"rows": len(rows_b), "boundary_rows": int(bnd.sum()), "mismatch_rows": 0,
+           "mismatch_boundary": 0, "near_tie_swaps": 0, "sum_within_error": 0}
+    unexplained = []
+    for r, (a, b) in enumerate(zip(rows_a, rows_b)):
+        a, b = list(a), list(b)
+        if a == b:
+            continue
+        out["mismatch_rows"] += 1
+        if bnd[r]:
+            out["mismatch_boundary"] += 1
+            continue
+        n = r % Nb + 1
+        sb = np.asarray(A_b[r], np.float64)
+        delta = float(np.abs(np.asarray(A_a[r], np.float64)[:n] - sb[:n]).max())
+        cut = float(sb[b].min())
+        diff = set(a) ^ set(b)
+        if len(a) == len(b) and all(abs(sb[J] - cut) <= 2 * delta for J in diff):
+            out["near_tie_swaps"] += 1
+            continue
+        _, cb, ca, thr, _ = diag_b[r]
+        if len(a) != len(b) and min(abs(cb - thr), abs(ca - thr)) <= 2 * n * delta:
+            out["sum_within_error"] += 1
+            continue
+        unexplained.append((r, a, b))
+    return out, unexplained
+
+
+def csr_rows(row_ptr, col_idx):
+    """Per-row lists of a CSR."""
+    rp = np.asarray(row_ptr)
+    ci = np.asarray(col_idx)
+    return [ci[rp[r]:rp[r + 1]].tolist() for r in range(len(rp) - 1)]
+
+
 def selection_accuracy(Q: torch.Tensor, K: torch.Tensor, S: int, B: int, tau: float,
                        protect_last: bool = True, strategy: str = "head",
                        layer: int = 0) -> Dict[str, object]:

@@ -26,6 +26,7 @@ import torch
 
 import long_context_prefill_estimate_b200 as rr
 import oracle
+from long_context_prefill_estimate_b200 import diagnostics
 import workloads
 
 pytestmark = pytest.mark.gpu
@@ -39,9 +40,7 @@ def _to(t, dev):
 
 
 def _csr_rows(rp, ci):
-    rp = np.asarray(rp)
-    ci = np.asarray(ci)
-    return [ci[rp[r]:rp[r + 1]].tolist() for r in range(len(rp) - 1)]
+    return diagnostics.csr_rows(rp, ci)
 
 
 def _boundary_rows(diag):
@@ -65,37 +64,8 @@ def _gpu_pipeline(w, t, dev, tau=None, protect_last=True, strategy="head", layer
 
 
 def _classify_masks(gpu_rows, rp_o, ci_o, diag, A_or, A_gpu):
-    """Compare the GPU's rows with the oracle's.  Row r of both lists is query block
-    I = r % Nb of a head (the lists start at a head boundary); A_or and A_gpu are the two
-    sides' scores of the same rows, [rows][Nb].  Returns the counts of the module docstring
-    and the rows no case explains."""
-    orc_rows = _csr_rows(rp_o, ci_o)
-    Nb = A_or.shape[-1]
-    bnd = _boundary_rows(diag)
-    out = {"rows": len(orc_rows), "boundary_rows": int(bnd.sum()), "mismatch_rows": 0,
-           "mismatch_boundary": 0, "near_tie_swaps": 0, "sum_within_error": 0}
-    unexplained = []
-    for r, (g, o) in enumerate(zip(gpu_rows, orc_rows)):
-        if g == o:
-            continue
-        out["mismatch_rows"] += 1
-        if bnd[r]:
-            out["mismatch_boundary"] += 1
-            continue
-        n = r % Nb + 1                      # causal blocks of the row
-        a_or = np.asarray(A_or[r], np.float64)
-        delta = float(np.abs(np.asarray(A_gpu[r], np.float64)[:n] - a_or[:n]).max())
-        cut = float(a_or[o].min())          # the oracle's k*-th score
-        diff = sorted(set(g) ^ set(o))
-        if len(g) == len(o) and all(abs(a_or[J] - cut) <= 2 * delta for J in diff):
-            out["near_tie_swaps"] += 1
-            continue
-        _, cb, ca, thr, _ = diag[r]
-        if len(g) != len(o) and min(abs(cb - thr), abs(ca - thr)) <= 2 * n * delta:
-            out["sum_within_error"] += 1
-            continue
-        unexplained.append((r, g, o))
-    return out, unexplained
+    """The row classes of the module docstring (GPU = side a, oracle = side b)."""
+    return diagnostics.classify_masks(gpu_rows, _csr_rows(rp_o, ci_o), diag, A_or, A_gpu, CUM_TOL)
 
 
 def _check_masks(gpu_rows, rp_o, ci_o, diag, A_or, A_gpu):
@@ -463,8 +433,6 @@ def test_full_size_layers(idx, w, cuda_device):
 def test_selection_accuracy_diagnostic(cuda_device):
     """RR selection vs the exact-mass (S = 1) selection: the GPU diagnostic equals the same
     metrics computed from oracle scores and oracle selections."""
-    from long_context_prefill_estimate_b200 import diagnostics
-
     w = workloads.get(1, H=4, Hkv=2, L=2048)
     t = workloads.generate(w)
     d = _to(t, cuda_device)

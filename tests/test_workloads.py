@@ -80,10 +80,12 @@ def test_bench_traffic_comes_from_the_matching_capture(tmp_path, monkeypatch):
     # a changed kernel source invalidates the capture
     fake = tmp_path / "repo"
     (fake / "profiles").mkdir(parents=True)
-    (fake / "long_context_prefill_estimate_b200" / "csrc").mkdir(parents=True)
-    shutil.copy(os.path.join(root, "profiles", "prefill_tc_llama3-8b-layer-L32k.md"), fake / "profiles")
-    src = os.path.join(root, "long_context_prefill_estimate_b200", "csrc", "rr_prefill_tc.cu")
-    (fake / "long_context_prefill_estimate_b200" / "csrc" / "rr_prefill_tc.cu").write_text(
-        open(src).read() + "\n// edited\n")
+    csrc = fake / "long_context_prefill_estimate_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    shutil.copy(os.path.join(root, "profiles", "prefill_tc_llama3-8b-layer-L32k.json"), fake / "profiles")
+    for name in ("rr_prefill_tc.cu", "rr_sm100.cuh"):
+        shutil.copy(os.path.join(root, "long_context_prefill_estimate_b200", "csrc", name), csrc)
     monkeypatch.setattr(bench, "ROOT", str(fake))
+    assert bench.prefill_traffic_per_launch(w32) == t32
+    (csrc / "rr_prefill_tc.cu").write_text((csrc / "rr_prefill_tc.cu").read_text() + "\n// edited\n")
     assert bench.prefill_traffic_per_launch(w32) is None
