@@ -1,7 +1,7 @@
-// Causal block-sparse attention over the selected blocks, two query tiles per CTA with their
-// softmax stages in alternation ("RRAttention: Dynamic Block Sparse Attention via Per-Head
-// Round-Robin Shifts for Long-Context Inference", Sec. 2.1 with the per-head CSR block lists
-// as the block selection matrix; Sec. 4.1: sparsity in prefill only).
+// Causal block-sparse attention over the selected blocks, two query tiles per CTA
+// ("RRAttention: Dynamic Block Sparse Attention via Per-Head Round-Robin Shifts for
+// Long-Context Inference", Sec. 2.1 with the per-head CSR block lists as the block selection
+// matrix; Sec. 4.1: sparsity in prefill only).
 //
 // Work unit: two query tiles of one query head, query blocks I and I-1 (128 rows each, B =
 // 128), one CTA per SM (the whole 512-column tensor memory).  Both tiles read the same KV head,
@@ -11,9 +11,8 @@
 // Per tile the chain is serial: S = Q K^T into the tile's S columns, softmax, P (bf16) written
 // over the first half of those columns, O += P V with P read from tensor memory, then the next
 // S into the same columns (the MMAs of one thread execute in order, so it never overwrites P
-// before the P V product has read it).  The two tiles alternate: while one tile's softmax runs,
-// the tensor core computes the other tile's P V and next S, so the exponentials of one tile
-// overlap the matrix products of the other.
+// before the P V product has read it).  While one tile's softmax runs, the tensor core can
+// compute the other tile's P V and next S.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer of Q (both tiles, once) and of the K tiles of the union (ring of
