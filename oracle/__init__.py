@@ -52,6 +52,8 @@ def _load():
     lib.rro_pool_keys.restype = None
     lib.rro_estimate.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, P]
     lib.rro_estimate.restype = I
+    lib.rro_xattn_estimate.argtypes = [P, P, I, I, I, I, I, I, I, I, P]
+    lib.rro_xattn_estimate.restype = I
     lib.rro_select.argtypes = [P, I, I, D, I, P, P, ctypes.c_int64, P]
     lib.rro_select.restype = I
     lib.rro_prefill_rows.argtypes = [P, P, P, I, I, I, I, I, P, P, D, P, ctypes.c_int64, P]
@@ -108,6 +110,21 @@ def estimate(Q, K, S: int, B: int, mode: int = HEAD_RR, layer: int = 0,
     rc = _load().rro_estimate(_ptr(q), _ptr(k), H, Hkv, L, d, S, B, mode, layer, h0, h1, _ptr(A))
     if rc:
         raise ValueError(f"oracle estimate rejected the arguments (code {rc})")
+    return A
+
+
+def xattn_estimate(Q, K, S: int, B: int, heads: Optional[Tuple[int, int]] = None) -> np.ndarray:
+    """XAttention's antidiagonal block importance A[H][Nb][Nb] (float64), the comparison
+    estimator; rows of heads outside ``heads`` are zero."""
+    q, k = _u16(Q), _u16(K)
+    H, L, d = q.shape
+    Hkv = k.shape[0]
+    Nb = L // B
+    A = np.zeros((H, Nb, Nb), np.float64)
+    h0, h1 = heads if heads is not None else (0, H)
+    rc = _load().rro_xattn_estimate(_ptr(q), _ptr(k), H, Hkv, L, d, S, B, h0, h1, _ptr(A))
+    if rc:
+        raise ValueError(f"oracle xattn_estimate rejected the arguments (code {rc})")
     return A
 
 

@@ -153,6 +153,65 @@ int rro_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, in
     return RRO_OK;
 }
 
+/* ---------------------------------------------------------------- XAttention estimate
+ * The comparison estimator of the pattern-discovery timing (RRAttention Sec. 4.2 "Runtime
+ * Efficiency", Fig. 3(b); RRAttention Sec. 2.2 and the XAttention card, "Summary" and "Key
+ * points"): inside every S x S sub-block of the attention logits (query stride i, key stride
+ * j) the entries on the antidiagonal, from lower-left (query iS+S-1, key jS) to upper-right
+ * (query iS, key jS+S-1), are summed; the sums are softmax-normalised over the key strides and
+ * aggregated into blocks, then the same Top-tau selection keeps the blocks.
+ * Readings where the pages are silent (the same as for the round-robin estimate):
+ *   x1 score a(i,j) = (1/(S sqrt d)) sum_{u<S} Q[iS+S-1-u] . K[jS+u], the mean of the S
+ *      antidiagonal logits q.k/sqrt(d) (the card's "sums", scaled like Sec. 3.2's 1/(S sqrt d));
+ *   x2 causality at stride granularity (j <= i), softmax over j in [0, i] (stride-level
+ *      softmax granularity, RRAttention Sec. 2.2);
+ *   x3 block score (S/B) * sum over the (B/S) x (B/S) sub-grid, as reading o4.
+ * A is [H][Nb][Nb]; rows of heads outside [h_begin, h_end) are not touched; J > I entries 0. */
+int rro_xattn_estimate(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, int d, int S,
+                       int B, int h_begin, int h_end, double *A) {
+    if (H <= 0 || Hkv <= 0 || H % Hkv || d <= 0 || S <= 0 || B <= 0 || B % S || L % B)
+        return RRO_EINVAL;
+    if (h_begin < 0 || h_end > H || h_begin > h_end) return RRO_EINVAL;
+    const long Ns = L / S, Nb = L / B, r = B / S;
+    const int G = H / Hkv;
+    const double scale = 1.0 / ((double)S * sqrt((double)d));
+    const double w = (double)S / (double)B;
+    const long nrows = (long)(h_end - h_begin) * Nb;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)Ns + 1);
+#pragma omp for schedule(dynamic, 1)
+        for (long row = 0; row < nrows; ++row) {
+            const int h = h_begin + (int)(row / Nb);
+            const long I = Nb - 1 - row % Nb; /* long rows first */
+            const int g = h / G;
+            double *Arow = A + ((long)h * Nb + I) * Nb;
+            for (long J = 0; J < Nb; ++J) Arow[J] = 0.0;
+            for (long i = I * r; i < (I + 1) * r; ++i) {
+                double m = -INFINITY;
+                for (long j = 0; j <= i; ++j) {
+                    double a = 0.0;
+                    for (int u = 0; u < S; ++u) {
+                        const uint16_t *q = Q + ((long)h * L + i * S + (S - 1 - u)) * d;
+                        const uint16_t *k = K + ((long)g * L + j * S + u) * d;
+                        for (int e = 0; e < d; ++e) a += bf16_to_double(q[e]) * bf16_to_double(k[e]);
+                    }
+                    p[j] = a * scale;
+                    if (p[j] > m) m = p[j];
+                }
+                double l = 0.0;
+                for (long j = 0; j <= i; ++j) {
+                    p[j] = exp(p[j] - m);
+                    l += p[j];
+                }
+                for (long j = 0; j <= i; ++j) Arow[j / r] += w * p[j] / l;
+            }
+        }
+        free(p);
+    }
+    return RRO_OK;
+}
+
 typedef struct {
     double a;
     int J;

@@ -27,6 +27,10 @@ MUTANTS = {
     "GQA group by modulo": ("const int g = h / G;\n            const long r", "const int g = h % Hkv;\n            const long r"),
     "softmax without max shift uses wrong sign": ("p[j] = exp(p[j] - m);", "p[j] = exp(m - p[j]);"),
     "transposed block accumulation": ("Arow[j / r] += w * p[j];", "Arow[(j / r) % (I + 1)] += w * p[i - j];"),
+    "xattn main diagonal": ("Q + ((long)h * L + i * S + (S - 1 - u)) * d;", "Q + ((long)h * L + i * S + u) * d;"),
+    "xattn drops 1/S": ("const double scale = 1.0 / ((double)S * sqrt((double)d));\n    const double w = (double)S / (double)B;\n    const long nrows = (long)(h_end - h_begin) * Nb;\n#pragma omp parallel\n    {\n        double *p = (double *)malloc(sizeof(double) * (size_t)Ns + 1);\n#pragma omp for schedule(dynamic, 1)",
+                        "const double scale = 1.0 / sqrt((double)d);\n    const double w = (double)S / (double)B;\n    const long nrows = (long)(h_end - h_begin) * Nb;\n#pragma omp parallel\n    {\n        double *p = (double *)malloc(sizeof(double) * (size_t)Ns + 1);\n#pragma omp for schedule(dynamic, 1)"),
+    "xattn stride causality j < i": ("for (long j = 0; j <= i; ++j) {\n                    double a = 0.0;", "for (long j = 0; j < i + (i == 0); ++j) {\n                    double a = 0.0;"),
     "diag cum_before reports cum_at": ("diag[1] = cum_before;", "diag[1] = cum;"),
     "diag threshold without tau": ("diag[3] = thr;", "diag[3] = T;"),
     "diag gap one past the cut": ("(kstar < n) ? buf[kstar - 1].a - buf[kstar].a",

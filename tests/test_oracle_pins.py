@@ -179,6 +179,77 @@ def test_estimate_reads_only_sampled_queries():
     assert d1[1].max() > 1e-6 and d1[0].max() == 0.0
 
 
+# ---------------------------------------------------------------- XAttention estimate
+def _golden_xattn():
+    out = []
+    with open(os.path.join(GOLDEN, "xattn_worked_example.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            q, k, a = line.split(";")
+            out.append(([float(v) for v in q.split()], [float(v) for v in k.split()],
+                        [float(v) for v in a.split()]))
+    return out
+
+
+@pytest.mark.parametrize("qv,kv,expected", _golden_xattn())
+def test_xattn_hand_worked(qv, kv, expected):
+    L = len(qv)
+    B = 2 if len(expected) == 4 else 4
+    Q = torch.tensor(qv, dtype=torch.bfloat16).reshape(1, L, 1)
+    K = torch.tensor(kv, dtype=torch.bfloat16).reshape(1, L, 1)
+    A = oracle.xattn_estimate(Q, K, S=2, B=B)
+    np.testing.assert_allclose(A.reshape(-1), expected, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("H,Hkv,L,d,B", [(2, 2, 128, 16, 16), (4, 2, 96, 8, 32)])
+def test_xattn_S1_is_exact_block_attention_mass(H, Hkv, L, d, B):
+    """S = 1: the antidiagonal of a 1 x 1 sub-block is the logit itself."""
+    Q, K = _bf16((H, L, d), 21), _bf16((Hkv, L, d), 22)
+    A = oracle.xattn_estimate(Q, K, S=1, B=B)
+    Nb, G = L // B, H // Hkv
+    for h in range(H):
+        P = _dense_causal_probs(Q[h].double(), K[h // G].double(), 1 / math.sqrt(d))
+        mass = P.reshape(Nb, B, Nb, B).sum(dim=(1, 3)) / B
+        np.testing.assert_allclose(A[h], mass.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("H,Hkv,L,d,S,B", [(2, 1, 64, 8, 4, 16), (3, 3, 48, 4, 2, 8), (2, 2, 64, 4, 8, 32)])
+def test_xattn_bruteforce_antidiagonals(H, Hkv, L, d, S, B):
+    """The full logits matrix (torch float64), the antidiagonal of every S x S sub-block taken
+    by flipping it left-right, the stride softmax and block sums written out directly."""
+    Q, K = _bf16((H, L, d), 23), _bf16((Hkv, L, d), 24)
+    A = oracle.xattn_estimate(Q, K, S=S, B=B)
+    Ns, Nb, G, r = L // S, L // B, H // Hkv, B // S
+    for h in range(H):
+        logits = (Q[h].double() @ K[h // G].double().T / math.sqrt(d)).numpy()
+        ref = np.zeros((Nb, Nb))
+        for i in range(Ns):
+            z = np.array([np.fliplr(logits[i * S:(i + 1) * S, j * S:(j + 1) * S]).trace() / S
+                          for j in range(i + 1)])
+            p = np.exp(z - z.max())
+            p /= p.sum()
+            for j in range(i + 1):
+                ref[i // r, j // r] += p[j] * S / B
+        np.testing.assert_allclose(A[h], ref, rtol=0, atol=1e-12)
+
+
+def test_xattn_equals_pooled_scores_for_constant_query_strides():
+    """Queries identical within each stride: every antidiagonal sum is q . (sum of the stride's
+    keys), the round-robin estimate's logit for that query."""
+    H, Hkv, L, d, S, B = 2, 1, 128, 16, 8, 32
+    qd = _bf16((H, L // S, d), 25)
+    Q = qd.repeat_interleave(S, dim=1).contiguous()
+    K = _bf16((Hkv, L, d), 26)
+    A = oracle.xattn_estimate(Q, K, S=S, B=B)
+    Kbar = K.double().reshape(Hkv, L // S, S, d).sum(2)
+    Ns, Nb, r = L // S, L // B, B // S
+    for h in range(H):
+        P = _dense_causal_probs(qd[h].double(), Kbar[0], 1 / (S * math.sqrt(d)))
+        mass = P.reshape(Nb, r, Nb, r).sum(dim=(1, 3)) / r
+        np.testing.assert_allclose(A[h], mass.numpy(), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- selection
 def _golden_select():
     out = []
