@@ -396,6 +396,7 @@ def run_ours(args):
     if rank == 0 and not args.quick:
         line["tau_sweep"] = tau_sweep(wl, step, st, ws, torch)
         line["dense_reference"] = dense_comparison(wl, Q, K, V, ws, rr, torch, st, ms_step)
+        line["pattern_discovery"] = pattern_discovery(wl, Q, K, ws, rr, torch, st, stage)
     line["e2e"] = e2e(w, wl, host, h0, layers, rr, torch, dev, args)
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
@@ -446,6 +447,37 @@ def tau_sweep(w, step, st, ws, torch):
                          "ms": ev[0].elapsed_time(ev[3]),
                          "prefill_ms": ev[2].elapsed_time(ev[3])}
     return out
+
+
+def pattern_discovery(w, Q, K, ws, rr, torch, st, stage):
+    """Pattern-discovery time (estimate + select) of the round-robin estimator (the timed
+    stages) and of XAttention's antidiagonal estimator on the same layer (the comparison of the
+    RRAttention page, Sec. 4.2 "Runtime Efficiency", Fig. 3(b)), with the density each keeps."""
+    res = {"rr_ms": stage["estimate_ms"] + stage["select_ms"]}
+    try:
+        A = torch.empty_like(ws.block_scores)
+        rp = torch.empty_like(ws.row_ptr)
+        ci = torch.empty_like(ws.col_idx)
+        nnz = torch.empty_like(ws.nnz)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        t_est, t_sel = [], []
+        for i in range(4):
+            ev[0].record(st)
+            rr.xattn_estimate(Q, K, w.S, w.B, out=A)
+            ev[1].record(st)
+            rr.select(A, w.tau, True, row_ptr=rp, col_idx=ci, nnz=nnz, workspace=ws.sel)
+            ev[2].record(st)
+            torch.cuda.synchronize()
+            if i:
+                t_est.append(ev[0].elapsed_time(ev[1]))
+                t_sel.append(ev[1].elapsed_time(ev[2]))
+        res["xattention_estimate_ms"] = statistics.median(t_est)
+        res["xattention_ms"] = statistics.median(t_est) + statistics.median(t_sel)
+        res["rr_time_saved"] = 1.0 - res["rr_ms"] / res["xattention_ms"]
+        res["xattention_density"] = int(nnz.item()) / (w.H * w.Nb * (w.Nb + 1) // 2)
+    except Exception as exc:  # sizes the comparison kernel does not cover
+        res["xattention_error"] = str(exc)[:200]
+    return res
 
 
 def dense_comparison(w, Q, K, V, ws, rr, torch, st, ms_sparse):

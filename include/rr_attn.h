@@ -99,6 +99,24 @@ rr_status_t rr_estimate_heads(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int
                               float *block_scores, void *workspace, size_t workspace_bytes,
                               rr_stream_t stream);
 
+/*
+ * rr_xattn_estimate -- XAttention's antidiagonal block importance, the estimator the paper
+ * compares pattern-discovery time against (Sec. 2.2; Sec. 4.2 "Runtime Efficiency", Fig. 3(b);
+ * the XAttention card, "Summary" and "Key points").  Not part of the RRAttention path.
+ *
+ * Inside every S x S sub-block of the logits (query stride i, key stride j) the antidiagonal
+ * from lower-left to upper-right is summed and scaled like the round-robin score:
+ *     z(h,i,j) = (1 / (S sqrt(d))) * sum_{u<S} Q[h][iS+S-1-u] . K[g(h)][jS+u],   j <= i,
+ * normalised by a softmax over j and aggregated exactly like rr_estimate's scores:
+ *     block_scores[h][I][J] = (S/B) * sum_{i in I} sum_{j in J, j <= i} p(h,i,j)
+ * ([H][L/B][L/B] float32, fully written, J > I entries 0), so rr_select applies unchanged.
+ * bf16 tensor-core products with fp32 accumulation over the S*d-long antidiagonal sums; softmax
+ * and block sums in fp32.  No workspace.  Supported: d in {64, 128}; B/S in {4, 8, 16, 32};
+ * (L/S) % 8 == 0; the common size rules above.
+ */
+rr_status_t rr_xattn_estimate(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L, int d,
+                              int S, int B, float *block_scores, rr_stream_t stream);
+
 /* Bytes of device workspace rr_select needs for H heads and Nb blocks per row. */
 size_t rr_select_workspace_bytes(int H, int Nb);
 
@@ -174,7 +192,8 @@ rr_status_t rr_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int 
 /*
  * rr_device_errors -- error bits the kernels recorded on the current device instead of
  * trapping: bit 0 producer, bit 1 MMA issuer, bit 2 softmax warps of rr_sparse_prefill, bit 3
- * a warp of rr_estimate's tensor-core kernel gave up a wait after about one second.  *flags
+ * a warp of rr_estimate's tensor-core kernel gave up a wait after about one second, bit 4 one of
+ * rr_xattn_estimate's.  *flags
  * (host) receives the bits; reset != 0 clears them.
  * Synchronous: waits for the device's preceding work.
  */

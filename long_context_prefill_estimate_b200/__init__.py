@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["RRAttnError", "lib", "library_path", "estimate", "select", "sparse_prefill",
+__all__ = ["RRAttnError", "lib", "library_path", "estimate", "xattn_estimate", "select", "sparse_prefill",
            "prefill", "validate_csr", "estimate_workspace_bytes", "select_workspace_bytes",
            "Workspace", "STRATEGIES", "EXPORTED_SYMBOLS", "device_errors", "default_chunks",
            "head_shard", "host_slices", "selftest_wait"]
@@ -31,7 +31,7 @@ library_path = os.path.join(_HERE, "librrattn.so")
 STRATEGIES = {"head": 0, "none": 1, "layer": 2, "hybrid": 3}
 
 EXPORTED_SYMBOLS = ("rr_estimate", "rr_estimate_strategy", "rr_estimate_heads",
-                    "rr_estimate_workspace_bytes",
+                    "rr_estimate_workspace_bytes", "rr_xattn_estimate",
                     "rr_select", "rr_select_workspace_bytes", "rr_select_noalloc",
                     "rr_sparse_prefill",
                     "rr_validate_csr", "rr_device_errors", "rr_selftest_wait", "rr_status_string",
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
     L.rr_estimate_strategy.restype = I
     L.rr_estimate_heads.argtypes = [P, P, I, I, I, I, I, I, I, I, I, P, P, Z, P]
     L.rr_estimate_heads.restype = I
+    L.rr_xattn_estimate.argtypes = [P, P, I, I, I, I, I, I, P, P]
+    L.rr_xattn_estimate.restype = I
     L.rr_select_workspace_bytes.argtypes = [I, I]
     L.rr_select_workspace_bytes.restype = Z
     L.rr_select.argtypes = [P, I, I, D, I, P, P, I64, P, P, Z, P]
@@ -161,6 +163,25 @@ def estimate(Q: torch.Tensor, K: torch.Tensor, S: int, B: int, strategy: str = "
     _check("rr_estimate", lib().rr_estimate_heads(
         _ptr(Q), _ptr(K), H, Hkv, L, d, S, B, STRATEGIES[strategy], layer, head_base, _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(Q.device)))
+    return out
+
+
+
+def xattn_estimate(Q: torch.Tensor, K: torch.Tensor, S: int, B: int,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """XAttention's antidiagonal block importance [H][L/B][L/B] (float32): the comparison
+    estimator of the pattern-discovery timing, selected with select() like estimate()'s."""
+    _need_cuda("rr_xattn_estimate", Q, torch.bfloat16)
+    _need_cuda("rr_xattn_estimate", K, torch.bfloat16)
+    H, L, d = Q.shape
+    Hkv = K.shape[0]
+    if K.shape != (Hkv, L, d):
+        raise RRAttnError("rr_xattn_estimate", 1, f"K shape {tuple(K.shape)} does not match Q {tuple(Q.shape)}")
+    Nb = L // B if B > 0 else 0
+    if out is None:
+        out = torch.empty((H, Nb, Nb), dtype=torch.float32, device=Q.device)
+    _check("rr_xattn_estimate", lib().rr_xattn_estimate(_ptr(Q), _ptr(K), H, Hkv, L, d, S, B, _ptr(out),
+                                                        _stream(Q.device)))
     return out
 
 

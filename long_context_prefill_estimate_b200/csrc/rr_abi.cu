@@ -33,6 +33,10 @@ rr_status_t launch_prefill_tc(const uint16_t *Q, const uint16_t *K, const uint16
 rr_status_t read_device_errors(unsigned *out, bool reset);
 rr_status_t read_estimate_errors(unsigned *out, bool reset);
 rr_status_t read_pp_errors(unsigned *out, bool reset);
+rr_status_t read_xattn_errors(unsigned *out, bool reset);
+bool xattn_supported(int d, int S, int B);
+rr_status_t launch_xattn(const uint16_t *Q, const uint16_t *K, int H, int Hkv, int L, int d, int S, int B,
+                         float *A, cudaStream_t st);
 rr_status_t selftest_wait(uint32_t timeout_us, uint32_t *result);
 
 #define RR_TRY(x)                       \
@@ -149,11 +153,12 @@ const char *rr_last_error(void) { return g_last_error; }
 rr_status_t rr_device_errors(uint32_t *flags, int reset) {
     clear_error();
     if (!flags) return set_error(RR_ERR_INVALID_ARG, "rr_device_errors: flags is NULL");
-    unsigned v = 0, ve = 0, vp = 0;
+    unsigned v = 0, ve = 0, vp = 0, vx = 0;
     rr_status_t s = read_device_errors(&v, reset != 0);
     if (s == RR_OK) s = read_estimate_errors(&ve, reset != 0);
     if (s == RR_OK) s = read_pp_errors(&vp, reset != 0);
-    *flags = v | ve | vp;
+    if (s == RR_OK) s = read_xattn_errors(&vx, reset != 0);
+    *flags = v | ve | vp | vx;
     return s;
 }
 
@@ -219,6 +224,25 @@ rr_status_t rr_estimate(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, 
                         size_t workspace_bytes, rr_stream_t stream) {
     return rr_estimate_strategy(Q, K, H, Hkv, L, d, S, B, RR_HEAD, 0, block_scores, workspace,
                                 workspace_bytes, stream);
+}
+
+rr_status_t rr_xattn_estimate(const rr_bf16_t *Q, const rr_bf16_t *K, int H, int Hkv, int L, int d,
+                              int S, int B, float *block_scores, rr_stream_t stream) {
+    static const char *fn = "rr_xattn_estimate";
+    const NvtxRange range(fn);
+    clear_error();
+    RR_TRY(check_common(fn, H, Hkv, L, d, B));
+    if (S <= 0 || S > B || B % S)
+        return set_error(RR_ERR_INVALID_ARG, "%s: stride S=%d must divide B=%d", fn, S, B);
+    if (!xattn_supported(d, S, B))
+        return set_error(RR_ERR_UNSUPPORTED, "%s: no kernel for d=%d B/S=%d", fn, d, B / S);
+    if ((L / S) % 8)
+        return set_error(RR_ERR_UNSUPPORTED, "%s: L/S=%d strides must be a multiple of 8", fn, L / S);
+    if (L == 0) return RR_OK;
+    RR_TRY(check_ptr(fn, "Q", Q));
+    RR_TRY(check_ptr(fn, "K", K));
+    RR_TRY(check_ptr(fn, "block_scores", block_scores));
+    return launch_xattn(Q, K, H, Hkv, L, d, S, B, block_scores, static_cast<cudaStream_t>(stream));
 }
 
 size_t rr_select_workspace_bytes(int H, int Nb) { return select_workspace_bytes(H, Nb); }

@@ -77,6 +77,22 @@ def test_estimate_rejections(L):
     assert _est(L, Len=0, q=0, k=0, out=0, ws=0) == 0   # empty problem: accepted, no launch
 
 
+def test_xattn_estimate_rejections(L):
+    def x(H=4, Hkv=2, Len=256, d=64, S=8, B=64, q=FAKE, k=FAKE, out=FAKE):
+        return L.rr_xattn_estimate(q, k, H, Hkv, Len, d, S, B, out, None)
+
+    assert x(H=3) == INVALID
+    assert x(d=96) == UNSUPPORTED
+    assert x(S=3) == INVALID
+    assert x(S=32) == UNSUPPORTED          # B/S = 2
+    assert x(S=1) == UNSUPPORTED           # B/S = 64: no kernel for XAttention
+    assert x(Len=64, S=16) == UNSUPPORTED  # L/S = 4
+    assert x(q=0) == INVALID
+    assert x(out=FAKE + 8) == INVALID
+    assert b"rr_xattn_estimate" in L.rr_last_error()
+    assert x(Len=0, q=0, k=0, out=0) == 0
+
+
 def test_estimate_heads_rejections(L):
     f = L.rr_estimate_heads
     ok = (FAKE, FAKE, 4, 2, 256, 64, 8, 64, 0, 0)

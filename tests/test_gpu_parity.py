@@ -430,6 +430,58 @@ def test_full_size_layers(idx, w, cuda_device):
     _check_output(O[idx_t[:, 0], idx_t[:, 1]].float().cpu().numpy(), O_ref)
 
 
+XATTN = [
+    ("tiny", workloads.get(0)),                                          # d = 64, S = 8, B = 64
+    ("llama-4k", workloads.get(1, L=4096)),                              # S = 16, B = 128
+    ("slash-8k", workloads.get(3, L=8192)),                              # several row groups
+    ("s32-b128", workloads.get(1, H=8, Hkv=2, L=4096, S=32)),            # B/S = 4
+    ("s4-b128-d64", workloads.get(0, H=4, Hkv=2, L=2048, d=64, S=4, B=128)),  # B/S = 32
+    ("ragged-rows", workloads.get(1, H=4, Hkv=1, L=2176, S=16, B=128)),  # 136 strides: a partial row group
+]
+
+
+@pytest.mark.parametrize("name,w", XATTN, ids=[x[0] for x in XATTN])
+def test_xattn_estimate_matches_oracle(name, w, cuda_device):
+    """XAttention's antidiagonal scores (the pattern-discovery comparison) against the oracle;
+    selection from them as for the round-robin scores."""
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    A = rr.xattn_estimate(d["Q"], d["K"], w.S, w.B)
+    rp, ci, nnz = rr.select(A, w.tau, True)
+    torch.cuda.synchronize()
+    assert rr.device_errors() == 0
+    A_gpu = A.cpu().numpy()
+    A_or = oracle.xattn_estimate(t["Q"], t["K"], w.S, w.B)
+    err = np.abs(A_gpu.astype(np.float64) - A_or).max()
+    assert err <= SCORE_TOL, f"block score error {err:.3e}"
+    assert np.abs(A_gpu.sum(-1) - 1.0).max() < 1e-4
+    n = int(nnz.item())
+    rp_h, ci_h = rp.cpu().numpy(), ci[:n].cpu().numpy()
+    rp_same, ci_same = oracle.select(A_gpu, w.tau, True)
+    assert np.array_equal(rp_h, rp_same) and np.array_equal(ci_h, ci_same)
+    rp_o, ci_o, dg = oracle.select(A_or, w.tau, True, diag=True)
+    H, Nb = w.H, w.Nb
+    _check_masks(_csr_rows(rp_h, ci_h), rp_o, ci_o, dg, A_or.reshape(H * Nb, Nb), A_gpu.reshape(H * Nb, Nb))
+
+
+def test_xattn_estimate_full_size_heads(cuda_device):
+    """The 32K Llama-shaped layer at full size: every head's scores on the GPU, two heads
+    recomputed by the oracle (its antidiagonal sums cost S times the round-robin scores)."""
+    w = workloads.get(1)
+    t = workloads.generate(w)
+    d = _to(t, cuda_device)
+    A = rr.xattn_estimate(d["Q"], d["K"], w.S, w.B)
+    torch.cuda.synchronize()
+    assert rr.device_errors() == 0
+    A_gpu = A.cpu().numpy()
+    assert np.abs(A_gpu.sum(-1) - 1.0).max() < 1e-4
+    assert not np.triu(A_gpu, 1).any()
+    for h in (0, 29):
+        A_or = oracle.xattn_estimate(t["Q"], t["K"], w.S, w.B, heads=(h, h + 1))
+        err = np.abs(A_gpu[h].astype(np.float64) - A_or[h]).max()
+        assert err <= SCORE_TOL, f"head {h}: block score error {err:.3e}"
+
+
 def test_selection_accuracy_diagnostic(cuda_device):
     """RR selection vs the exact-mass (S = 1) selection: the GPU diagnostic equals the same
     metrics computed from oracle scores and oracle selections."""

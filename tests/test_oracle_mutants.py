@@ -14,18 +14,22 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "rr_oracle.c")
 
 MUTANTS = {
-    "logit scale drops 1/S": ("1.0 / ((double)S * sqrt((double)d))", "1.0 / sqrt((double)d)"),
+    "logit scale drops 1/S": ("double *p) {\n    const double scale = 1.0 / ((double)S * sqrt((double)d));",
+                              "double *p) {\n    const double scale = 1.0 / sqrt((double)d);"),
     "stride causality j < i": ("for (long j = 0; j <= i; ++j) {\n        const double *kb",
                                "for (long j = 0; j < i + (i == 0); ++j) {\n        const double *kb"),
     "head offset shifted": ("case RRO_HEAD_RR: return h % S;", "case RRO_HEAD_RR: return (h + 1) % S;"),
-    "pool keeps first key only": ("for (int u = 0; u < S; ++u)", "for (int u = 0; u < 1; ++u)"),
-    "block weight 1/B": ("const double w = (double)S / (double)B;", "const double w = 1.0 / (double)B;"),
+    "pool keeps first key only": ("for (int u = 0; u < S; ++u) {\n                const uint16_t *k = K + ((long)g * L + j * S + u) * d;",
+                                  "for (int u = 0; u < 1; ++u) {\n                const uint16_t *k = K + ((long)g * L + j * S + u) * d;"),
+    "block weight 1/B": ("rro_pool_keys(K, Hkv, L, d, S, Kbar);\n    const double w = (double)S / (double)B;",
+                         "rro_pool_keys(K, Hkv, L, d, S, Kbar);\n    const double w = 1.0 / (double)B;"),
     "select strict >": ("if (cum >= thr)", "if (cum > thr)"),
     "tie-break reversed": ("return (u->J > v->J) - (u->J < v->J);", "return (u->J < v->J) - (u->J > v->J);"),
     "prefill drops diagonal key": ("k < (J + 1) * B && k <= t; ++k) {\n                    const uint16_t *kr",
                                    "k < (J + 1) * B && k < t + (k == 0); ++k) {\n                    const uint16_t *kr"),
     "GQA group by modulo": ("const int g = h / G;\n            const long r", "const int g = h % Hkv;\n            const long r"),
-    "softmax without max shift uses wrong sign": ("p[j] = exp(p[j] - m);", "p[j] = exp(m - p[j]);"),
+    "softmax without max shift uses wrong sign": ("p[j] = exp(p[j] - m);\n        l += p[j];\n    }\n    for (long j = 0; j <= i; ++j) p[j] /= l;",
+                                                  "p[j] = exp(m - p[j]);\n        l += p[j];\n    }\n    for (long j = 0; j <= i; ++j) p[j] /= l;"),
     "transposed block accumulation": ("Arow[j / r] += w * p[j];", "Arow[(j / r) % (I + 1)] += w * p[i - j];"),
     "xattn main diagonal": ("Q + ((long)h * L + i * S + (S - 1 - u)) * d;", "Q + ((long)h * L + i * S + u) * d;"),
     "xattn drops 1/S": ("const double scale = 1.0 / ((double)S * sqrt((double)d));\n    const double w = (double)S / (double)B;\n    const long nrows = (long)(h_end - h_begin) * Nb;\n#pragma omp parallel\n    {\n        double *p = (double *)malloc(sizeof(double) * (size_t)Ns + 1);\n#pragma omp for schedule(dynamic, 1)",
