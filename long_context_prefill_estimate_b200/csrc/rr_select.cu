@@ -163,6 +163,14 @@ __device__ __forceinline__ float warp_sum_f(float v) {
     return v;
 }
 
+// acc += x when the bit pattern of x is >= mid: one compare and one predicated add (the add
+// on the FMA pipe, not a select on the integer pipe, which the search otherwise saturates).
+__device__ __forceinline__ void add_if_at_least(float &acc, float x, uint32_t mid) {
+    asm("{\n\t.reg .pred p;\n\tsetp.ge.u32 p, %1, %2;\n\t@p add.f32 %0, %0, %3;\n\t}"
+        : "+f"(acc)
+        : "r"(__float_as_uint(x)), "r"(mid), "f"(x));
+}
+
 // Fixed-point value of a non-negative float with bit pattern b, on the grid of a row whose
 // maximum has biased exponent E (E >= 1): b's value times 2^(176 - E), truncated.
 __device__ __forceinline__ long long to_fixed(uint32_t b, int E) {
@@ -208,8 +216,8 @@ __device__ __forceinline__ void select_row_warp(const float *__restrict__ a, int
         float p0 = 0.f, p1 = 0.f;
 #pragma unroll
         for (int k = 0; k < NS; k += 2) {
-            if (__float_as_uint(v[k]) >= mid) p0 += v[k];
-            if (__float_as_uint(v[k + 1]) >= mid) p1 += v[k + 1];
+            add_if_at_least(p0, v[k], mid);
+            add_if_at_least(p1, v[k + 1], mid);
         }
         const float p = warp_sum_f(p0 + p1);
         bool ge;
@@ -300,39 +308,60 @@ __global__ void __launch_bounds__(256, 4)
     }
 }
 
+// One CTA: the counts in chunks of 4096 (four consecutive rows per thread, one 16-byte load when
+// aligned), a block-wide exclusive scan per chunk, a running carry between chunks.
 __global__ void __launch_bounds__(1024)
     scan_counts_kernel(const int *__restrict__ counts, long nrows, int32_t *__restrict__ row_ptr,
                        int64_t *__restrict__ nnz_out) {
     __shared__ long warp_tot[32];
+    __shared__ long s_carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long per = (nrows + 1023) / 1024;
-    const long r0 = tid * per, r1 = min(r0 + per, nrows);
-    long local = 0;
-    for (long r = r0; r < r1; ++r) local += counts[r];
-    long x = local;
-    for (int o = 1; o < 32; o <<= 1) {
-        const long y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_tot[warp] = x;
+    if (tid == 0) s_carry = 0;
     __syncthreads();
-    if (warp == 0) {
-        long t = warp_tot[lane];
-        for (int o = 1; o < 32; o <<= 1) {
-            const long y = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += y;
+    for (long c0 = 0; c0 < nrows; c0 += 4096) {
+        const long r0 = c0 + 4L * tid;
+        int cv[4];
+        if (r0 + 3 < nrows && (r0 & 3) == 0) {
+            const int4 q = *reinterpret_cast<const int4 *>(counts + r0);
+            cv[0] = q.x, cv[1] = q.y, cv[2] = q.z, cv[3] = q.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cv[k] = r0 + k < nrows ? counts[r0 + k] : 0;
         }
-        warp_tot[lane] = t;
+        const long local = (long)cv[0] + cv[1] + cv[2] + cv[3];
+        long x = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_tot[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            long t = warp_tot[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
+            }
+            warp_tot[lane] = t;
+        }
+        __syncthreads();
+        const long carry = s_carry;
+        long at = carry + (warp ? warp_tot[warp - 1] : 0) + x - local;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (r0 + k < nrows) {
+                row_ptr[r0 + k] = (int32_t)at;
+                at += cv[k];
+            }
+        __syncthreads();  // every thread has read s_carry and warp_tot
+        if (tid == 1023) s_carry = carry + warp_tot[31];
+        __syncthreads();
     }
-    __syncthreads();
-    long at = (warp ? warp_tot[warp - 1] : 0) + x - local;
-    for (long r = r0; r < r1; ++r) {
-        row_ptr[r] = (int32_t)at;
-        at += counts[r];
-    }
-    if (tid == 1023) {
-        row_ptr[nrows] = (int32_t)warp_tot[31];
-        if (nnz_out) *nnz_out = warp_tot[31];
+    if (tid == 0) {
+        row_ptr[nrows] = (int32_t)s_carry;
+        if (nnz_out) *nnz_out = s_carry;
     }
 }
 
