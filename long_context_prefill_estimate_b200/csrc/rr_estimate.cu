@@ -7,12 +7,13 @@
 //   estimate_tc_kernel     one CTA per (KV head g, chunk of hc of g's query heads, group of
 //                          QB consecutive query blocks).  Its 128 rows are the sampled
 //                          queries Q[h][i*S + off(h)] of those heads and blocks (QB * hc * r
-//                          of them, r = B/S), staged once into shared memory in the tensor
-//                          core's 128-byte-swizzled layout.  Pooled keys arrive by TMA in
-//                          tiles of 64 strides; S = Qhat (Kbar_hi + Kbar_lo)^T (fp32-grade
-//                          logits) goes to one of two TMEM buffers.  96 KB of shared memory
-//                          and 128 TMEM columns per CTA: two CTAs share an SM, so the
-//                          softmax of one overlaps the MMAs and loads of the other.  Two passes over the
+//                          of them, r = B/S), staged once into TMEM (the MMA's A operand, read
+//                          from tensor memory, so shared memory feeds only the key tiles).
+//                          Pooled keys arrive by TMA in tiles of 64 strides (a ring of three);
+//                          S = Qhat (Kbar_hi + Kbar_lo)^T (fp32-grade logits) goes to one of
+//                          two TMEM buffers.  96 KB of shared memory and 256 TMEM columns per
+//                          CTA: two CTAs share an SM, so the softmax of one overlaps the MMAs
+//                          and loads of the other.  Two passes over the
 //                          tiles: the first finds each row's max and sum of exp2 over the
 //                          causal strides j <= i; the second recomputes S, normalises exactly,
 //                          sums each key block's r strides and reduces over the r rows of each
@@ -21,8 +22,8 @@
 // For r <= 32 the r rows of a (head, query block) lie in one warp and are reduced with
 // shuffles; for r = 64 or 128 they span r/32 warps, whose sums meet in shared memory behind
 // bounded mbarrier waits (a fixed summation order, so the result is deterministic).
-// Warp roles: 0 TMA producer and TMEM allocation, 1 MMA issuer, 2-3 staging only, 4-7 softmax
-// (thread = row = TMEM lane).  Every wait is bounded; a timeout sets a device error bit.
+// Warp roles: 0 TMA producer and TMEM allocation, 1 MMA issuer, 2-3 idle, 4-7 staging of the
+// sampled rows, then softmax (thread = row = TMEM lane).  Every wait is bounded; a timeout sets a device error bit.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -89,10 +90,9 @@ struct EstTcParams {
 template <int D>
 struct EstTcCfg {
     static constexpr int DC = D / 64;
-    static constexpr uint32_t Q_BYTES = kRows * D * 2;
     static constexpr uint32_t T_BYTES = kTileN * D * 2;  // one hi or lo key tile
-    static constexpr int NS = D == 128 ? 2 : 4;          // stages of (hi, lo) tiles
-    static constexpr uint32_t BAR_OFF = Q_BYTES + NS * 2 * T_BYTES;
+    static constexpr int NS = D == 128 ? 3 : 6;          // stages of (hi, lo) tiles
+    static constexpr uint32_t BAR_OFF = NS * 2 * T_BYTES;  // the sampled rows live in TMEM
     // k_full[NS], k_empty[NS], s_full[2], s_free[2], fin, red_full[2], red_empty[2]
     static constexpr uint32_t NBAR = 2 * NS + 9;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
@@ -109,10 +109,11 @@ __global__ void __launch_bounds__(256, 2)
     constexpr int NBT = kTileN / R;  // key blocks per tile
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sQ = smem_u32(base);
-    auto sHi = [&](int s) { return sQ + C::Q_BYTES + s * 2 * C::T_BYTES; };
-    auto sLo = [&](int s) { return sQ + C::Q_BYTES + s * 2 * C::T_BYTES + C::T_BYTES; };
-    const uint32_t sBar = sQ + C::BAR_OFF;
+    const uint32_t sK = smem_u32(base);  // ring of (hi, lo) key tiles
+    auto sHi = [&](int s) { return sK + s * 2 * C::T_BYTES; };
+    auto sLo = [&](int s) { return sK + s * 2 * C::T_BYTES + C::T_BYTES; };
+    constexpr uint32_t Q_COL = 2 * kTileN;  // TMEM columns of the sampled rows (bf16 pairs)
+    const uint32_t sBar = sK + C::BAR_OFF;
     auto k_full = [&](int s) { return sBar + 8u * s; };
     auto k_empty = [&](int s) { return sBar + 8u * (NS + s); };
     auto s_full = [&](int b) { return sBar + 8u * (2 * NS + b); };
@@ -154,33 +155,43 @@ __global__ void __launch_bounds__(256, 2)
         sm100::fence_mbar_init();
     }
     if (warp == 0) {
-        sm100::tmem_alloc(smem_u32(tmem_slot), 2 * kTileN);
+        sm100::tmem_alloc(smem_u32(tmem_slot), 4 * kTileN);
         sm100::tmem_relinquish();
     }
-    // Stage the sampled rows: row rho = qb*RB + hh*r + ii samples stride i = (I0+qb)*r + ii of
-    // head g*G + hci*hc + hh.  16-byte unit u of the row goes to the 128-byte-swizzled slot
-    // (u % 8) ^ (rho % 8) of column chunk u / 8.
-    constexpr int UPR = D / 8;
-    for (int x = tid; x < kRows * UPR; x += 256) {
-        const int rho = x / UPR, u = x % UPR;
-        uint4 v = make_uint4(0, 0, 0, 0);
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // Stage the sampled rows into TMEM (the MMA's A operand): row rho = qb*RB + hh*r + ii, the
+    // sample of stride i = (I0+qb)*r + ii of head g*G + hci*hc + hh, in lane rho, two bf16 per
+    // column.  Warps 4-7 own the four lane quadrants.
+    if (warp >= 4) {
+        const int rho = (warp & 3) * 32 + lane;
+        uint32_t w[D / 2];
         if (rho < nrows) {
             const int qb = rho / p.RB, rr_ = rho % p.RB, hh = rr_ / R, ii = rr_ % R;
             const int h = g * p.G + hci * p.hc + hh;
             const long i = (long)(I0 + qb) * R + ii;
             const long pos = i * p.S + rr_offset(p.head_base + h, p.S, p.mode, p.layer);
-            v = __ldg(reinterpret_cast<const uint4 *>(p.Q + ((long)h * p.L + pos) * D) + u);
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.Q + ((long)h * p.L + pos) * D);
+#pragma unroll
+            for (int u = 0; u < D / 8; ++u) {
+                const uint4 v = __ldg(src + u);
+                w[4 * u] = v.x, w[4 * u + 1] = v.y, w[4 * u + 2] = v.z, w[4 * u + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < D / 2; ++k) w[k] = 0u;
         }
-        const uint32_t dst = sQ + (u / 8) * (kRows * 128) + rho * 128 + (((u % 8) ^ (rho & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                     "r"(v.w)
-                     : "memory");
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc)
+            sm100::tmem_st32(trow + Q_COL + cc * 32, *reinterpret_cast<const uint32_t(*)[32]>(w + cc * 32));
+        sm100::tmem_wait_st();
     }
-    sm100::fence_proxy_async_smem();  // the tensor core reads what these threads wrote
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
     const int nq = 2 * nT;  // tile visits over both passes
 
     if (warp == 0) {
@@ -224,16 +235,14 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk >> 2, w4 = kk & 3;
-                    const uint64_t ad = sm100::smem_desc_sw128(sQ + c * kRows * 128 + w4 * 32, 16, 1024);
                     const uint64_t bd = sm100::smem_desc_sw128(sHi(s) + c * kTileN * 128 + w4 * 32, 16, 1024);
-                    sm100::mma_ss(tmem + b * kTileN, ad, bd, C::IDESC, kk > 0);
+                    sm100::mma_ts(tmem + b * kTileN, tmem + Q_COL + kk * 8, bd, C::IDESC, kk > 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk >> 2, w4 = kk & 3;
-                    const uint64_t ad = sm100::smem_desc_sw128(sQ + c * kRows * 128 + w4 * 32, 16, 1024);
                     const uint64_t bd = sm100::smem_desc_sw128(sLo(s) + c * kTileN * 128 + w4 * 32, 16, 1024);
-                    sm100::mma_ss(tmem + b * kTileN, ad, bd, C::IDESC, 1);
+                    sm100::mma_ts(tmem + b * kTileN, tmem + Q_COL + kk * 8, bd, C::IDESC, 1);
                 }
                 sm100::mma_commit(k_empty(s));
                 sm100::mma_commit(s_full(b));
@@ -364,7 +373,7 @@ __global__ void __launch_bounds__(256, 2)
     if (warp == 0) {
         __syncwarp();  // lane 0 ran the producer; dealloc is warp-collective
         sm100::tc_fence_after();
-        sm100::tmem_dealloc(tmem, 2 * kTileN);
+        sm100::tmem_dealloc(tmem, 4 * kTileN);
     }
 }
 
