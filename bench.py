@@ -65,11 +65,17 @@ def profile_record(name):
     return rec
 
 
+# committed DRAM counter record of the prefill kernel that serves each block size
+PREFILL_RECORDS = {128: "prefill_pp_llama3-8b-layer-L32k"}
+
+
 def prefill_traffic_per_launch(w):
     """DRAM bytes (read + write) per prefill launch from the committed capture, scaled by L
     from the captured layer to this one (Q, K, V and O all grow linearly with L at fixed heads
-    and d).  None when the kernel changed since the capture or the layer shape differs."""
-    rec = profile_record("prefill_tc_llama3-8b-layer-L32k")
+    and d).  None when the kernel changed since the capture, no capture covers this block
+    size, or the layer shape differs."""
+    name = PREFILL_RECORDS.get(w.B)
+    rec = profile_record(name) if name else None
     if rec is None:
         return None
     if (w.H, w.Hkv, w.d, w.B) != tuple(rec["shape"][k] for k in ("H", "Hkv", "d", "B")):

@@ -61,10 +61,11 @@ def test_bench_flop_accounting():
 
 
 def test_bench_traffic_comes_from_the_matching_capture(tmp_path, monkeypatch):
-    # the roofline's DRAM traffic is the committed ncu capture at 32K scaled by L, for the
-    # captured shape only, and only while the kernel source matches the capture's hash
+    # the roofline's DRAM traffic is a committed ncu record at 32K scaled by L, for the
+    # captured shape only, and only while every source the record names hashes as recorded
+    import hashlib
+    import json
     import os
-    import shutil
     import sys
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -72,20 +73,33 @@ def test_bench_traffic_comes_from_the_matching_capture(tmp_path, monkeypatch):
     import bench
 
     w32, w128 = workloads.get(1), workloads.get(2)
-    t32 = bench.prefill_traffic_per_launch(w32)
-    if t32 is None:  # the capture predates the current kernel source: nothing to check
-        return
-    assert bench.prefill_traffic_per_launch(w128) == 4 * t32
-    assert bench.prefill_traffic_per_launch(workloads.get(0)) is None      # other shape
-    # a changed kernel source invalidates the capture
     fake = tmp_path / "repo"
     (fake / "profiles").mkdir(parents=True)
-    csrc = fake / "long_context_prefill_estimate_b200" / "csrc"
-    csrc.mkdir(parents=True)
-    shutil.copy(os.path.join(root, "profiles", "prefill_tc_llama3-8b-layer-L32k.json"), fake / "profiles")
-    for name in ("rr_prefill_tc.cu", "rr_sm100.cuh"):
-        shutil.copy(os.path.join(root, "long_context_prefill_estimate_b200", "csrc", name), csrc)
+    src = fake / "kernel.cu"
+    src.write_text("// kernel source\n")
+    rec = {"shape": {"H": w32.H, "Hkv": w32.Hkv, "L": w32.L, "d": w32.d, "B": w32.B},
+           "dram_bytes_read": 3.0e8, "dram_bytes_write": 1.0e8,
+           "sources": {"kernel.cu": hashlib.sha256(src.read_bytes()).hexdigest()[:16]}}
+    name = bench.PREFILL_RECORDS[w32.B]
+    (fake / "profiles" / (name + ".json")).write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(fake))
-    assert bench.prefill_traffic_per_launch(w32) == t32
-    (csrc / "rr_prefill_tc.cu").write_text((csrc / "rr_prefill_tc.cu").read_text() + "\n// edited\n")
+    assert bench.prefill_traffic_per_launch(w32) == 4.0e8
+    assert bench.prefill_traffic_per_launch(w128) == 4 * 4.0e8
+    assert bench.prefill_traffic_per_launch(workloads.get(0)) is None      # other shape
+    src.write_text("// kernel source\n// edited\n")                       # changed kernel
     assert bench.prefill_traffic_per_launch(w32) is None
+
+
+def test_committed_counter_records_name_existing_sources():
+    import glob
+    import json
+    import os
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    recs = [r for r in glob.glob(os.path.join(root, "profiles", "*.json")) if "mask_parity" not in r]
+    assert recs
+    for r in recs:
+        rec = json.load(open(r))
+        assert rec["sources"] and "command" in rec and "shape" in rec, r
+        for path, digest in rec["sources"].items():
+            assert os.path.exists(os.path.join(root, path)) and len(digest) == 16, (r, path)
