@@ -78,21 +78,35 @@ __device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
 }
 
 // The merged, ascending union of two ascending block lists; next() yields each block once
-// with the lists that hold it.
+// with the lists that hold it.  Each list's next two entries are held in registers and the
+// entry after them is loaded when one is consumed, so a load is issued a union step before
+// its value is needed and the MMA issuer does not wait on global memory between steps.
 struct UnionWalk {
     const int32_t *a, *b;
     int na, nb, ia, ib;
+    int a0, a1, b0, b1;  // a[ia], a[ia+1], b[ib], b[ib+1]; INT_MAX past the end
     __device__ UnionWalk(const int32_t *a_, int na_, const int32_t *b_, int nb_)
-        : a(a_), b(b_), na(na_), nb(nb_), ia(0), ib(0) {}
+        : a(a_), b(b_), na(na_), nb(nb_), ia(0), ib(0) {
+        a0 = na > 0 ? __ldg(a) : INT_MAX;
+        a1 = na > 1 ? __ldg(a + 1) : INT_MAX;
+        b0 = nb > 0 ? __ldg(b) : INT_MAX;
+        b1 = nb > 1 ? __ldg(b + 1) : INT_MAX;
+    }
     __device__ __forceinline__ bool next(int &J, bool &inA, bool &inB) {
-        if (ia >= na && ib >= nb) return false;
-        const int ja = ia < na ? __ldg(a + ia) : INT_MAX;
-        const int jb = ib < nb ? __ldg(b + ib) : INT_MAX;
-        J = min(ja, jb);
-        inA = ja == J;
-        inB = jb == J;
-        ia += inA;
-        ib += inB;
+        if (a0 == INT_MAX && b0 == INT_MAX) return false;
+        J = min(a0, b0);
+        inA = a0 == J;
+        inB = b0 == J;
+        if (inA) {
+            ++ia;
+            a0 = a1;
+            a1 = ia + 1 < na ? __ldg(a + ia + 1) : INT_MAX;
+        }
+        if (inB) {
+            ++ib;
+            b0 = b1;
+            b1 = ib + 1 < nb ? __ldg(b + ib + 1) : INT_MAX;
+        }
         return true;
     }
 };
@@ -266,28 +280,36 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
             // ---------------------------------------------------------------- MMA issuer
             bool ok = sm100::mbar_wait(q_full, 0);
             sm100::tc_fence_after();
+            // shared-memory descriptors of the operand bases, built once: an MMA step only adds
+            // the step's byte offset >> 4 to the start-address field (every address is below
+            // 256 KB, so the 14-bit field never carries into the next one).  The issuing thread
+            // runs only a few instructions between MMAs: the tensor core queues almost nothing
+            // ahead of the MMA it executes, so every instruction in between can leave it idle.
+            const uint64_t dQ0 = sm100::smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t dQ1 = sm100::smem_desc_sw128(sQ + C::Q_BYTES, 16, 1024);
+            const uint64_t dK0 = sm100::smem_desc_sw128(sK, 16, 1024);
+            const uint64_t dV0 = sm100::smem_desc_sw128(sV, kBlk * 128, 1024);
             // P V of tile x for the union block held in V slot vs; n = blocks of x done so far
             auto issue_pv = [&](int x, int vs, int n) -> bool {
                 if (!sm100::mbar_wait(p_full(x), n & 1)) return false;
                 sm100::tc_fence_after();
+                const uint64_t bd0 = dV0 + ((vs * C::T_BYTES) >> 4);
+                const uint32_t dcol = tmem + C::O_COL + x * D, acol = tmem + x * kBlk;
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t bd =
-                        sm100::smem_desc_sw128(sV + vs * C::T_BYTES + kk * 16 * 128, kBlk * 128, 1024);
-                    sm100::mma_ts(tmem + C::O_COL + x * D, tmem + x * kBlk + kk * 8, bd, C::IDESC_PV,
+                for (int kk = 0; kk < kBlk / 16; ++kk)
+                    sm100::mma_ts(dcol, acol + kk * 8, bd0 + ((kk * 16 * 128) >> 4), C::IDESC_PV,
                                   (n > 0 || kk > 0));
-                }
                 return true;
             };
             auto issue_s = [&](int x, int ks) {
-                const uint32_t q = sQ + x * C::Q_BYTES;
+                const uint64_t ad0 = x ? dQ1 : dQ0;
+                const uint64_t bd0 = dK0 + ((ks * C::T_BYTES) >> 4);
+                const uint32_t dcol = tmem + x * kBlk;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk >> 2, w = kk & 3;
-                    const uint64_t ad = sm100::smem_desc_sw128(q + c * kRowsPP * 128 + w * 32, 16, 1024);
-                    const uint64_t bd =
-                        sm100::smem_desc_sw128(sK + ks * C::T_BYTES + c * kBlk * 128 + w * 32, 16, 1024);
-                    sm100::mma_ss(tmem + x * kBlk, ad, bd, C::IDESC_S, kk > 0);
+                    sm100::mma_ss(dcol, ad0 + ((c * kRowsPP * 128 + w * 32) >> 4),
+                                  bd0 + ((c * kBlk * 128 + w * 32) >> 4), C::IDESC_S, kk > 0);
                 }
                 sm100::mma_commit(s_full(x));
             };
