@@ -3,10 +3,13 @@
 // Long-Context Inference", Sec. 2.1 with the per-head CSR block lists as the block selection
 // matrix; Sec. 4.1: sparsity in prefill only).
 //
-// One CTA per (query head h, query block I): a 128-row query tile (for B = 64 the upper 64
-// rows are padding that is computed and never stored).  The CTA walks only the CSR entries
-// of row h*Nb + I, each key block as 64-key sub-blocks.  Two CTAs share an SM, so each SM
-// sub-partition runs two independent softmax streams.  Warp roles (224 threads):
+// B = 64 layers.  One CTA per (query head h, pair of query blocks 2p and 2p+1): a 128-row
+// query tile whose rows 0-63 are block 2p and rows 64-127 block 2p+1, so no tensor-core row
+// is padding.  The CTA walks the ascending union of the two blocks' CSR lists, one 64-key
+// block per step; each softmax warp's 32 rows lie in one half, and a warp whose block's list
+// lacks the step's key block writes P = 0 for it (masking the whole block, no exponentials).
+// Two CTAs share an SM, so each SM sub-partition runs two independent softmax streams.
+// Warp roles (224 threads):
 //   warp 0      TMA producer of Q (once) and of the K sub-tiles, into a ring of two or more
 //               (128-byte swizzle, mbarrier transaction counts); L2 prefetch of upcoming
 //               sub-tiles; TMEM allocation / release.
@@ -70,6 +73,22 @@ __device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
 constexpr int kBM = 128;  // query rows per CTA
 constexpr int kSub = 64;  // keys per sub-block: the unit of S, P and the K/V pipeline
 
+// The two query blocks' CSR lists as bitmaps over the key blocks (shared memory, filled once):
+// the steps of the CTA are the set bits of their union in ascending order.
+constexpr int kBmWords = kMaxL / 64 / 32;  // bitmap words per list, enough for any layer B = 64 allows
+
+// The union block after `cur` (-1 when there is none).
+__device__ __forceinline__ int next_block(const uint32_t *bmL, const uint32_t *bmH, int W, int cur) {
+    int w = (cur + 1) >> 5;
+    if (w >= W) return -1;
+    uint32_t m = (bmL[w] | bmH[w]) & (~0u << ((cur + 1) & 31));
+    while (m == 0) {
+        if (++w >= W) return -1;
+        m = bmL[w] | bmH[w];
+    }
+    return (w << 5) + __ffs(m) - 1;
+}
+
 template <int D, int BN>
 struct TcCfg {
     static constexpr int DC = D / 64;       // 64-element (128-byte) column chunks
@@ -78,7 +97,7 @@ struct TcCfg {
     static constexpr uint32_t SUB_BYTES = kSub * D * 2;  // one K or V sub-tile
     // Two CTAs per SM: each may use 113 KB of shared memory (1024 bytes of that are
     // alignment slack, 256 barriers); the rest holds K and V sub-tile rings.
-    static constexpr int SLOTS = (int)((113u * 1024u - 1024u - 256u - Q_BYTES) / SUB_BYTES);
+    static constexpr int SLOTS = (int)((113u * 1024u - 1024u - 256u - 8u * kBmWords - Q_BYTES) / SUB_BYTES);
     static constexpr int NK = SLOTS / 2 > 4 ? 4 : SLOTS / 2;
     static constexpr int NV = NK;
     static constexpr int PF = 8;  // sub-blocks prefetched into L2 ahead of the shared-memory loads
@@ -86,7 +105,8 @@ struct TcCfg {
     // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full, s_free, p_full[2],
     // o_bar, fin
     static constexpr uint32_t NBAR = 1 + 2 * NK + 2 * NV + 6;
-    static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16;
+    static constexpr uint32_t BM_OFF = BAR_OFF + NBAR * 8 + 16;  // the two list bitmaps
+    static constexpr uint32_t SMEM = BM_OFF + 8 * kBmWords;
     // at least 80 KB so that a third CTA never fits on an SM (3 x 80 KB > 228 KB): with two
     // CTAs of 256 TMEM columns each, a TMEM allocation never waits
     static constexpr uint32_t SMEM_LAUNCH = SMEM + 1024 > 80u * 1024u ? SMEM + 1024 : 80u * 1024u;
@@ -96,7 +116,7 @@ struct TcCfg {
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t IDESC_S = sm100::idesc_bf16(kBM, kSub, false);
     static constexpr uint32_t IDESC_PV = sm100::idesc_bf16(kBM, D, true);
-    static_assert(BN % kSub == 0, "key blocks are whole sub-blocks");
+    static_assert(BN == kSub && 2 * BN == kBM, "two 64-row query blocks per tile, one 64-key block per step");
     static_assert(NK >= 2, "need at least two K and two V sub-tiles");
     static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM + 1024 <= 113u * 1024u, "two CTAs per SM");
@@ -129,18 +149,28 @@ __global__ void __launch_bounds__(224, 2)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + C::BAR_OFF + C::NBAR * 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // Launch order: KV group by KV group, and inside a group query blocks from the longest
-    // CSR rows down with the group's heads adjacent.  CTAs resident at the same time then
-    // stream one KV head's K/V, which stays in L2.
-    const int G = H / Hkv;
+    // Launch order: KV group by KV group, and inside a group pairs of query blocks from the
+    // longest CSR rows down with the group's heads adjacent.  CTAs resident at the same time
+    // then stream one KV head's K/V, which stays in L2.
+    const int G = H / Hkv, NPR = (Nb + 1) / 2;
     const long lin = blockIdx.x;
-    const int g = (int)(lin / ((long)G * Nb));
-    const int within = (int)(lin % ((long)G * Nb));
-    const int I = Nb - 1 - within / G;
+    const int g = (int)(lin / ((long)G * NPR));
+    const int within = (int)(lin % ((long)G * NPR));
+    const int I_lo = 2 * (NPR - 1 - within / G), I_hi = I_lo + 1;  // I_hi == Nb: no upper block
     const int h = g * G + within % G;
-    const long crow = (long)h * Nb + I;
-    const int e0 = row_ptr[crow];
-    const int nsub = (row_ptr[crow + 1] - e0) * NSB;  // sub-block t: block e0 + t / NSB, half t % NSB
+    const long crow = (long)h * Nb + I_lo;
+    const int eL = row_ptr[crow], nL = row_ptr[crow + 1] - eL;
+    const int eH = I_hi < Nb ? row_ptr[crow + 1] : 0;
+    const int nH = I_hi < Nb ? row_ptr[crow + 2] - eH : 0;
+    const int32_t *listL = col_idx + eL, *listH = col_idx + eH;
+    uint32_t *bmL = reinterpret_cast<uint32_t *>(base + C::BM_OFF), *bmH = bmL + kBmWords;
+    const int W = (Nb + 31) / 32;
+    for (int w = threadIdx.x; w < 2 * W; w += blockDim.x) (w < W ? bmL[w] : bmH[w - W]) = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nL + nH; i += blockDim.x) {
+        const int J = i < nL ? __ldg(listL + i) : __ldg(listH + i - nL);
+        atomicOr((i < nL ? bmL : bmH) + (J >> 5), 1u << (J & 31));
+    }
 
     if (threadIdx.x == 64) {
         sm100::mbar_init(q_full, 1);
@@ -168,7 +198,11 @@ __global__ void __launch_bounds__(224, 2)
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    auto key_row = [&](int t) { return g * L + __ldg(col_idx + e0 + t / NSB) * BN + (t % NSB) * kSub; };
+    // steps: the blocks of the union (every warp counts them, 32 bitmap words per lane step)
+    int nsub = 0;
+    for (int w = lane; w < W; w += 32) nsub += __popc(bmL[w] | bmH[w]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nsub += __shfl_xor_sync(0xffffffffu, nsub, o);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -178,26 +212,24 @@ __global__ void __launch_bounds__(224, 2)
             sm100::prefetch_tmap(&tmV);
             sm100::mbar_arrive_expect_tx(q_full, C::Q_BYTES);
             for (int c = 0; c < C::DC; ++c)
-                sm100::tma_load_2d(sQ + c * kBM * 128, &tmQ, c * 64, h * L + I * BN, q_full);
-            for (int t = 0; t < nsub && t < C::PF; ++t) {
-                const int y = key_row(t);
+                sm100::tma_load_2d(sQ + c * kBM * 128, &tmQ, c * 64, h * L + I_lo * BN, q_full);
+            int ja = -1, J = -1;  // prefetch cursor (PF blocks ahead) and load cursor
+            for (int t = 0; t < C::PF && (ja = next_block(bmL, bmH, W, ja)) >= 0; ++t)
                 for (int c = 0; c < C::DC; ++c) {
-                    sm100::tma_prefetch_2d(&tmK, c * 64, y);
-                    sm100::tma_prefetch_2d(&tmV, c * 64, y);
+                    sm100::tma_prefetch_2d(&tmK, c * 64, g * L + ja * BN);
+                    sm100::tma_prefetch_2d(&tmV, c * 64, g * L + ja * BN);
                 }
-            }
             int issued = 0;
             bool ok = true;
             for (int t = 0; t < nsub; ++t) {
-                if (t + C::PF < nsub) {
-                    const int y = key_row(t + C::PF);
+                if (ja >= 0 && (ja = next_block(bmL, bmH, W, ja)) >= 0)
                     for (int c = 0; c < C::DC; ++c) {
-                        sm100::tma_prefetch_2d(&tmK, c * 64, y);
-                        sm100::tma_prefetch_2d(&tmV, c * 64, y);
+                        sm100::tma_prefetch_2d(&tmK, c * 64, g * L + ja * BN);
+                        sm100::tma_prefetch_2d(&tmV, c * 64, g * L + ja * BN);
                     }
-                }
                 const int s = t % NK;
-                const int y = key_row(t);
+                J = next_block(bmL, bmH, W, J);
+                const int y = g * L + J * BN;
                 if (!sm100::mbar_wait(k_empty(s), ((t / NK) & 1) ^ 1)) {  // S_{t-NK} has completed
                     ok = false;
                     break;
@@ -218,11 +250,12 @@ __global__ void __launch_bounds__(224, 2)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------------- V producer
-            int issued = 0;
+            int issued = 0, J = -1;
             bool ok = true;
             for (int t = 0; t < nsub; ++t) {
                 const int s = t % NV;
-                const int y = key_row(t);
+                J = next_block(bmL, bmH, W, J);
+                const int y = g * L + J * BN;
                 if (!sm100::mbar_wait(v_empty(s), ((t / NV) & 1) ^ 1)) {  // P_{t-NV} V_{t-NV} has completed
                     ok = false;
                     break;
@@ -291,13 +324,17 @@ __global__ void __launch_bounds__(224, 2)
         // -------------------------------------------------------------------- softmax
         // warps 3-6; a warp may only touch TMEM lanes 32*(warp % 4) .. +31
         const int r = (warp & 3) * 32 + lane;  // query row within the tile = TMEM lane
-        const long qpos = (long)I * BN + r;
+        const bool upper = r >= BN;             // the warp's rows are all in one half
+        const int Iown = upper ? I_hi : I_lo, rb = r - (upper ? BN : 0);
+        const long qpos = (long)I_lo * BN + r;
         const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        // A CSR row is ascending with J <= I, so only its last block can be the diagonal one.
-        const int tdiag = (nsub > 0 && __ldg(col_idx + e0 + nsub / NSB - 1) == I) ? nsub - NSB : nsub;
+        const uint32_t *bmOwn = upper ? bmH : bmL;
+        int J = -1;
         for (int t = 0; t < nsub; ++t) {
+            J = next_block(bmL, bmH, W, J);
+            const bool mine = (bmOwn[J >> 5] >> (J & 31)) & 1u;  // warp-uniform
             ok = __all_sync(0xffffffffu, sm100::mbar_wait(s_full, t & 1));
             if (!ok) break;
             sm100::tc_fence_after();
@@ -308,11 +345,13 @@ __global__ void __launch_bounds__(224, 2)
             // S_t is in registers: the MMA warp may write S_{t+1}
             sm100::tc_fence_before();
             sm100::mbar_arrive(s_free);
-            if (t >= tdiag) {  // diagonal block: key k0 + i of the block is visible iff k0 + i <= r
-                const int k0 = (t - tdiag) * kSub;
+            // keys i > lim are masked: none (lim = 63), those after the row on its diagonal block,
+            // or all of a block this half's list does not hold (lim = -1)
+            const int lim = !mine ? -1 : (J == Iown ? rb : kSub - 1);
+            if (lim < kSub - 1) {
 #pragma unroll
                 for (int i = 0; i < kSub; ++i)
-                    if (k0 + i > r) sr[i] = __float_as_uint(-INFINITY);
+                    if (i > lim) sr[i] = __float_as_uint(-INFINITY);
             }
             // row max: four chains of three-input maxima
             float mq[4];
@@ -405,7 +444,7 @@ __global__ void __launch_bounds__(224, 2)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16(__uint_as_float(rg[2 * i]) * inv, __uint_as_float(rg[2 * i + 1]) * inv);
-                if (r < BN) {
+                if (!upper || I_hi < Nb) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
@@ -438,7 +477,7 @@ rr_status_t launch_tc(const uint16_t *Q, const uint16_t *K, const uint16_t *V, i
     if (e != cudaSuccess)
         return set_error(RR_ERR_CUDA, "rr_sparse_prefill: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     const int Nb = L / BN;
-    dim3 grid((unsigned)((long)H * Nb));
+    dim3 grid((unsigned)((long)H * ((Nb + 1) / 2)));
     kern<<<grid, 224, smem, st>>>(mq, mk, mv, O, row_ptr, col_idx, H, Hkv, L, Nb,
                                   scale * 1.4426950408889634f);
     return check_launch("rr_sparse_prefill: prefill_tc_kernel");

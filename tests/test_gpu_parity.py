@@ -96,6 +96,9 @@ SMALL = [
     ("s32-b128", workloads.get(1, H=8, Hkv=2, L=4096, S=32)),      # B/S = 4: two blocks per tile
     ("s16-b64", workloads.get(0, L=2176, S=16, B=64)),              # B/S = 4 at B = 64
     ("s4-b128", workloads.get(0, H=4, Hkv=2, L=2048, d=64, S=4, B=128)),  # B/S = 32
+    # B = 64 at d = 128 with an odd number of query blocks: the last pair of 64-row blocks has
+    # no upper block
+    ("b64-d128-odd", workloads.get(1, H=4, Hkv=2, L=64 * 37, d=128, S=8, B=64)),
 ]
 
 
