@@ -7,14 +7,14 @@
 // query tile whose rows 0-63 are block 2p and rows 64-127 block 2p+1, so no tensor-core row
 // is padding.  The CTA walks the ascending union of the two blocks' CSR lists, one 64-key
 // block per step; each softmax warp's 32 rows lie in one half, and a warp whose block's list
-// lacks the step's key block writes P = 0 for it (masking the whole block, no exponentials).
+// lacks the step's key block masks that whole block (P = 0 for its rows).
 // Two CTAs share an SM, so each SM sub-partition runs two independent softmax streams.
 // Warp roles (224 threads):
-//   warp 0      TMA producer of Q (once) and of the K sub-tiles, into a ring of two or more
+//   warp 0      TMA producer of Q (once) and of the K tiles, into a ring of two or more
 //               (128-byte swizzle, mbarrier transaction counts); L2 prefetch of upcoming
-//               sub-tiles; TMEM allocation / release.
-//   warp 1      TMA producer of the V sub-tiles (its own ring, so K loads never queue behind
-//               a V slot that is still being read).
+//               tiles; TMEM allocation / release.
+//   warp 1      TMA producer of the V tiles (its own ring, so K loads never queue behind a V
+//               slot that is still being read).
 //   warp 2      MMA issuer (one thread): S_t = Q K_t^T (both operands in shared memory) into
 //               the single S buffer as soon as the softmax has loaded S_{t-1}, so S_t is
 //               computed while the softmax works on S_{t-1}; then O += P_t V_t with P_t read
