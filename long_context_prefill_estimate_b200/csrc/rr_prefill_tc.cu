@@ -92,7 +92,6 @@ __device__ __forceinline__ int next_block(const uint32_t *bmL, const uint32_t *b
 template <int D, int BN>
 struct TcCfg {
     static constexpr int DC = D / 64;       // 64-element (128-byte) column chunks
-    static constexpr int NSB = BN / kSub;   // sub-blocks per key block
     static constexpr uint32_t Q_BYTES = kBM * D * 2;
     static constexpr uint32_t SUB_BYTES = kSub * D * 2;  // one K or V sub-tile
     // Two CTAs per SM: each may use 113 KB of shared memory (1024 bytes of that are
@@ -129,7 +128,7 @@ __global__ void __launch_bounds__(224, 2)
                       const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
                       int H, int Hkv, int L, int Nb, float scale_log2) {
     using C = TcCfg<D, BN>;
-    constexpr int NK = C::NK, NV = C::NV, NSB = C::NSB;
+    constexpr int NK = C::NK, NV = C::NV;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_u32(base);
