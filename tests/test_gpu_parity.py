@@ -99,6 +99,10 @@ SMALL = [
     # B = 64 at d = 128 with an odd number of query blocks: the last pair of 64-row blocks has
     # no upper block
     ("b64-d128-odd", workloads.get(1, H=4, Hkv=2, L=64 * 37, d=128, S=8, B=64)),
+    # B = 128 with an odd number of query blocks: the last CTA holds block 0 alone (no second
+    # tile), beside two-tile CTAs of the same heads
+    ("b128-d128-odd", workloads.get(1, H=4, Hkv=2, L=128 * 37, S=16)),
+    ("b128-d64-odd", workloads.get(0, H=2, Hkv=1, L=128 * 11, d=64, S=8, B=128)),
 ]
 
 
